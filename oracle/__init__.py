@@ -1,0 +1,208 @@
+"""CPU oracle for the Hadamard-rotation + block-quantization paths.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline / reference leg may import this package.  The product
+library (``nvfp4_quantization_group_b200``) never imports it, and it never
+imports the product library: the two share no code.
+
+The arithmetic lives in ``hq_oracle.c`` (plain single-threaded C, IEEE
+binary32, no contraction); this module compiles it with gcc on first use and
+wraps it with numpy arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hq_oracle.c")
+_LIB = os.path.join(_HERE, "libhq_oracle.so")
+_CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile hq_oracle.c into libhq_oracle.so (skipped when up to date)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            i64 = ctypes.c_int64
+            L.hqo_e4m3_encode.argtypes = [ctypes.c_float]
+            L.hqo_e4m3_encode.restype = ctypes.c_uint8
+            L.hqo_e4m3_decode.argtypes = [ctypes.c_uint8]
+            L.hqo_e4m3_decode.restype = ctypes.c_float
+            L.hqo_e2m1_encode.argtypes = [ctypes.c_float]
+            L.hqo_e2m1_encode.restype = ctypes.c_uint8
+            L.hqo_e2m1_decode.argtypes = [ctypes.c_uint8]
+            L.hqo_e2m1_decode.restype = ctypes.c_float
+            L.hqo_encode_array.argtypes = [ctypes.c_int, P, P, i64]
+            L.hqo_encode_array.restype = None
+            L.hqo_exp.argtypes = [ctypes.c_float]
+            L.hqo_exp.restype = ctypes.c_float
+            L.hqo_exp_array.argtypes = [P, P, i64]
+            L.hqo_exp_array.restype = None
+            L.hqo_fwht.argtypes = [P, ctypes.c_int]
+            L.hqo_fwht.restype = None
+            L.hqo_cat_rotate_fp8.argtypes = [P, i64, ctypes.c_int, P, i64, ctypes.c_int, i64,
+                                             ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, i64, P]
+            L.hqo_cat_rotate_fp8.restype = ctypes.c_int
+            L.hqo_swiglu_fp8_k128.argtypes = [ctypes.c_int, P, i64, i64, P, P, P]
+            L.hqo_swiglu_fp8_k128.restype = ctypes.c_int
+            L.hqo_group_rht_quant.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_uint16, ctypes.c_uint,
+                                              P, P, P, P, P, P, P, P, P, P]
+            L.hqo_group_rht_quant.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+# ------------------------------------------------------------------ scalars
+def e4m3_encode(v: float) -> int:
+    return int(lib().hqo_e4m3_encode(float(v)))
+
+
+def e4m3_decode(c: int) -> float:
+    return float(lib().hqo_e4m3_decode(int(c)))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(lib().hqo_e2m1_encode(float(v)))
+
+
+def e2m1_decode(c: int) -> float:
+    return float(lib().hqo_e2m1_decode(int(c)))
+
+
+E4M3, E2M1 = 0, 1
+
+
+def encode_array(fmt: int, x: np.ndarray) -> np.ndarray:
+    """Per-element E4M3 (fmt 0) or E2M1 nibble (fmt 1) codes of FP32 values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    lib().hqo_encode_array(fmt, _ptr(x), _ptr(out), x.size)
+    return out
+
+
+def exp_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(x)
+    lib().hqo_exp_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def fwht(v: np.ndarray) -> np.ndarray:
+    """Unnormalised Sylvester Hadamard butterfly of an FP32 vector (copy)."""
+    v = np.array(v, dtype=np.float32, copy=True)
+    lib().hqo_fwht(_ptr(v), v.size)
+    return v
+
+
+# -------------------------------------------------------------- operations
+ROWMAJOR, TRANSPOSED = 0, 1
+
+
+def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=None,
+                   scale_layout=ROWMAJOR, scale_ld=None, want_pre=False):
+    """Concat (a | b) per group, optional 128-point Hadamard, FP8 1x128 quant.
+
+    a, b: uint16 BF16 bit arrays; a_width = a.shape[-1] (b may be None).
+    Returns (codes [M, G*128] uint8, scales, pre or None).
+    """
+    a = np.ascontiguousarray(a, dtype=np.uint16)
+    a_w = int(a.shape[-1])
+    a_rs = a_row_stride if a_row_stride is not None else G * a_w
+    if b is not None:
+        b = np.ascontiguousarray(b, dtype=np.uint16)
+        b_w = int(b.shape[-1])
+        b_rs = b_row_stride if b_row_stride is not None else G * b_w
+    else:
+        b_w, b_rs = 0, 0
+    out = np.empty((M, G * 128), dtype=np.uint8)
+    if scale_layout == ROWMAJOR:
+        scales = np.empty((M, G), dtype=np.float32)
+        ld = G
+    else:
+        ld = scale_ld if scale_ld is not None else M
+        scales = np.zeros((G, ld), dtype=np.float32)
+    pre = np.empty((M, G * 128), dtype=np.float32) if want_pre else None
+    rc = lib().hqo_cat_rotate_fp8(_ptr(a), a_rs, a_w, _ptr(b), b_rs, b_w, M, G, hadamard_n,
+                                  _ptr(out), _ptr(scales), scale_layout, ld, _ptr(pre))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, scales, pre
+
+
+NONE_BF16, NONE_F32, SWIGLU_F32 = 0, 1, 2
+
+
+def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False):
+    """K128 FP8 quantization of BF16/FP32 rows or of SiLU(gate) * up."""
+    x = np.ascontiguousarray(x)
+    out = np.empty((M, K_out), dtype=np.uint8)
+    scales = np.empty((M, K_out // 128), dtype=np.float32)
+    pre = np.empty((M, K_out), dtype=np.float32) if want_pre else None
+    rc = lib().hqo_swiglu_fp8_k128(mode, _ptr(x), M, K_out, _ptr(out), _ptr(scales), _ptr(pre))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, scales, pre
+
+
+ROWWISE, COLWISE = 1, 2
+
+
+def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=False):
+    """Grouped RHT16 + NVFP4 cast.  x: uint16 BF16 bits [M, K].
+
+    Returns a dict with row_codes [M, K/2], row_sf [M, K/16], col_codes
+    [M*K/2], col_sf [M*K/16] (sections concatenated, each [K, M_s/...]),
+    amax_row, amax_col, sdec_row, sdec_col [S] and, if asked, the
+    pre-rounding values row_pre [M, K] / col_pre [M*K].
+    """
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    M, K = x.shape
+    splits = np.ascontiguousarray(split_rows, dtype=np.int64)
+    S = splits.size
+    r = {}
+    if flags & ROWWISE:
+        r["row_codes"] = np.empty((M, K // 2), dtype=np.uint8)
+        r["row_sf"] = np.empty((M, K // 16), dtype=np.uint8)
+        r["amax_row"] = np.empty(S, dtype=np.float32)
+        r["sdec_row"] = np.empty(S, dtype=np.float32)
+        if want_pre:
+            r["row_pre"] = np.empty((M, K), dtype=np.float32)
+    if flags & COLWISE:
+        r["col_codes"] = np.empty(M * K // 2, dtype=np.uint8)
+        r["col_sf"] = np.empty(M * K // 16, dtype=np.uint8)
+        r["amax_col"] = np.empty(S, dtype=np.float32)
+        r["sdec_col"] = np.empty(S, dtype=np.float32)
+        if want_pre:
+            r["col_pre"] = np.empty(M * K, dtype=np.float32)
+    g = r.get
+    rc = lib().hqo_group_rht_quant(_ptr(x), M, K, _ptr(splits), S, sign_mask, flags,
+                                   _ptr(g("row_codes")), _ptr(g("row_sf")), _ptr(g("col_codes")),
+                                   _ptr(g("col_sf")), _ptr(g("amax_row")), _ptr(g("amax_col")),
+                                   _ptr(g("sdec_row")), _ptr(g("sdec_col")), _ptr(g("row_pre")),
+                                   _ptr(g("col_pre")))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return r

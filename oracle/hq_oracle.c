@@ -1,0 +1,501 @@
+/*
+ * hq_oracle.c -- plain, slow, single-threaded CPU reference for the three
+ * Hadamard-rotation + block-quantization paths.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may load this file's library.  It shares no code, header,
+ * table or constant generator with the CUDA library.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC
+ * (FLT_EVAL_METHOD == 0 on x86-64: every float operation below is one IEEE
+ * binary32 operation rounded to nearest even; fmaf() is the fused multiply-add
+ * with a single rounding).  No multiply-add is contracted unless fmaf() is
+ * written out.
+ *
+ * Sources (page title, then the part of the page):
+ *  [QMOE]  onnxruntime PR #33644, "Add opt-in activation_quantization=
+ *          dynamic_fp8 to com.microsoft::QMoE", Description: consecutive K128
+ *          groups, saturating nearest-even E4M3, scale max(amax,1e-10) *
+ *          float32(1/448), FP32 normalization, FP32 SiLU/SwiGLU before the
+ *          second quantizer, and the review note that NaN must stay NaN.
+ *  [DSA]   TensorRT-LLM PR #15158 "[#13061][bugfix] Add rotate_activation to
+ *          DSA fused_cat_fp8 path", Summary and code flow: cat([pe, nope]) ->
+ *          rotate_activation (orthonormal Hadamard) -> fp8_quantize_1x128,
+ *          scales transposed; the review thread's (Hq).(Hk) = q.k argument.
+ *  [GRP]   TransformerEngine PR #2564 "[NVFP4][MOE] Bug Fix for NVFP4 Grouped
+ *          Quant", Greptile summary and changed-file list: grouped row cast +
+ *          column Hadamard transform + cast with scale factors, per MoE split.
+ *  [FUS]   TransformerEngine PR #2555 review comments (cast.cpp, quantizer.cpp):
+ *          split_section % 128 fusion rule, rht_matrix, rowwise output needs
+ *          no RHT, the RHT'd columnwise output is the transposed layout.
+ *
+ * Where the pages leave a step open, the reading taken is stated beside it
+ * and listed in the repository's design notes.  Function names start hqo_.
+ *
+ * Pins (tests/test_oracle_pins.py): E4M3/E2M1 encoders against exact
+ * nearest-even brute force over the bit-field grids and torch's e4m3 cast;
+ * the butterfly against scipy's Sylvester matrix; FP8 scales/codes against
+ * the printed rule with exact rational quotients and crafted midpoint cases;
+ * exp against FP64; NVFP4 against exact block-scale/code brute force,
+ * dequantization bounds and the inverse-rotation round trip.
+ * Parity unpinned (readings the pages leave open, each moving results only
+ * inside the 2^-20 midpoint window or the 1e-5 rotation tolerance): the
+ * ascending butterfly stage order, and the operation order of the NVFP4
+ * block scale ((a_b / 6) * S_enc) and of enc = S_enc / sf.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- helpers */
+
+static float bf16_value(uint16_t bits)
+{
+    /* BF16 is the upper half of an IEEE binary32 word. */
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------ E4M3 */
+/*
+ * E4M3 ("e4m3fn"): 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no
+ * infinities, NaN = S.1111.111, largest finite 448 = 1.75 * 2^8, smallest
+ * normal 2^-6, subnormals m * 2^-9 (m = 1..7).  [QMOE] asks for saturating
+ * nearest-even conversion.  Reading: round the exact binary32 value to the
+ * nearest E4M3 value, ties to the even code; a magnitude that rounds above 448
+ * (and +-inf) saturates to +-448; the sign of zero is kept; NaN stays NaN.
+ */
+float hqo_e4m3_decode(uint8_t c)
+{
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    float v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexpf((float)m, -9);
+    else
+        v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+    return sign ? -v : v;
+}
+
+uint8_t hqo_e4m3_encode(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    if (isnan(v))
+        return sign | 0x7F;
+    float a = fabsf(v);
+    if (a >= 448.0f)                     /* everything from 448 up saturates */
+        return sign | 0x7E;
+    if (a == 0.0f)
+        return sign;
+    int ex;
+    frexpf(a, &ex);                      /* a = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                      /* a in [2^E, 2^(E+1)) */
+    if (E < -6)
+        E = -6;                          /* subnormal range keeps 2^-9 spacing */
+    float quantum = ldexpf(1.0f, E - 3); /* spacing of E4M3 values near a */
+    float n = nearbyintf(a / quantum);   /* a / quantum is exact; RNE to integer */
+    float r = n * quantum;               /* exact E4M3 value, r <= 448 */
+    if (r == 0.0f)
+        return sign;
+    if (r < ldexpf(1.0f, -6))            /* subnormal code: r = m * 2^-9 */
+        return sign | (uint8_t)(r / ldexpf(1.0f, -9));
+    int rex;
+    frexpf(r, &rex);
+    int RE = rex - 1;
+    int m = (int)((r / ldexpf(1.0f, RE) - 1.0f) * 8.0f);
+    return sign | (uint8_t)(((RE + 7) << 3) | m);
+}
+
+/* ------------------------------------------------------------------ E2M1 */
+/*
+ * E2M1 (the element type of NVFP4): magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6},
+ * code = sign << 3 | index into that list.  The pages name NVFP4 but no
+ * detail.  Reading: the OCP FP4 E2M1 format, round to nearest with ties to the
+ * even code, magnitudes from 6 up saturate to 6, the sign of zero is kept.
+ * NaN has no code and is outside the contract (returns 0xFF as a marker).
+ */
+float hqo_e2m1_decode(uint8_t nib)
+{
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    float v = mag[nib & 7];
+    return (nib & 8) ? -v : v;
+}
+
+uint8_t hqo_e2m1_encode(float v)
+{
+    if (isnan(v))
+        return 0xFF;
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    float a = fabsf(v);
+    if (a >= 6.0f)
+        return sign | 7;
+    /* spacing of the grid: 0.5 below 2, 1 in [2, 4), 2 in [4, 6] */
+    float quantum = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    float r = nearbyintf(a / quantum) * quantum;
+    for (uint8_t i = 0; i < 8; ++i)
+        if (hqo_e2m1_decode(i) == r)
+            return sign | i;
+    return 0xFF; /* unreachable */
+}
+
+void hqo_encode_array(int fmt, const float *in, uint8_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = fmt == 0 ? hqo_e4m3_encode(in[i]) : hqo_e2m1_encode(in[i]);
+}
+
+/* -------------------------------------------------------------- Hadamard */
+/*
+ * Unnormalised Sylvester-ordered Walsh-Hadamard transform, H[i][j] =
+ * (-1)^popcount(i & j), applied in place as butterflies: for h = 1, 2, 4, ...,
+ * n/2 (ascending) and every i with (i & h) == 0, (a, b) -> (a + b, a - b).
+ * The pages fix only "Hadamard rotation" ([DSA]) and "random Hadamard
+ * transform" with a 16x16 rht_matrix ([FUS]); the Sylvester order, the
+ * ascending stage order and a single scaling multiply at the end are the
+ * reading taken here.
+ */
+void hqo_fwht(float *v, int n)
+{
+    for (int h = 1; h < n; h <<= 1)
+        for (int i = 0; i < n; ++i)
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+/* 1/sqrt(128) = 2^-3.5 rounded to binary32 (0x3DB504F3); the pages scale the
+ * 128-point rotation by 1/sqrt(128) so that it is orthonormal. */
+static float c128(void)
+{
+    uint32_t u = 0x3DB504F3u;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ---------------------------------------------------------------- FP8 1xN */
+/*
+ * One group of n values -> n E4M3 codes and one FP32 scale, as [QMOE] states:
+ *   amax = max |y|                      (fmaxf, so a NaN element is skipped)
+ *   s    = max(amax, 1e-10f) * float32(1/448)
+ *   q_i  = e4m3(y_i / s)                (IEEE binary32 division)
+ * The page says "FP32 div.full normalization" and notes that the choice of
+ * division changes codes by one ulp at FP8 midpoints.  Reading: correctly
+ * rounded IEEE division.  `pre`, when given, receives y_i / s (the value that
+ * is rounded to E4M3).
+ */
+static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, float *pre)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        amax = fmaxf(amax, fabsf(y[i]));
+    const float inv448 = 1.0f / 448.0f; /* binary32 constant, 0x3B124925 */
+    float s = fmaxf(amax, 1e-10f) * inv448;
+    for (int i = 0; i < n; ++i) {
+        float t = y[i] / s;
+        if (pre)
+            pre[i] = t;
+        q[i] = hqo_e4m3_encode(t);
+    }
+    *scale = s;
+}
+
+/*
+ * DSA indexer prep [DSA]: for token t and group (head) g the 128-vector is
+ * a[t, g, 0:a_width] followed by b[t, g, 0:b_width] (pe first, then nope),
+ * optionally rotated by the orthonormal 128-point Hadamard (Sylvester
+ * butterfly, then * 1/sqrt(128)), then quantized as one 1x128 FP8 group.
+ * Element (t, g, j) of a is a[t * a_row_stride + g * a_width + j]; b likewise.
+ * Output codes: out[(t * G + g) * 128 + j].  Scales: scale_layout 0 (row
+ * major) puts group (t, g) at scales[t * G + g]; layout 1 (transposed, as the
+ * indexer stores them) at scales[g * scale_ld + t].
+ * Returns 0, or -1 for arguments this reference does not accept.
+ */
+int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
+                       const uint16_t *b, int64_t b_row_stride, int b_width,
+                       int64_t M, int G, int hadamard_n,
+                       uint8_t *out, float *scales, int scale_layout, int64_t scale_ld,
+                       float *pre)
+{
+    if (a_width < 0 || b_width < 0 || a_width + b_width != 128 || (b_width > 0 && !b))
+        return -1;
+    if (hadamard_n != 0 && hadamard_n != 128)
+        return -1;
+    const float c = c128();
+    float v[128];
+    for (int64_t t = 0; t < M; ++t)
+        for (int g = 0; g < G; ++g) {
+            for (int j = 0; j < a_width; ++j)
+                v[j] = bf16_value(a[t * a_row_stride + (int64_t)g * a_width + j]);
+            for (int j = 0; j < b_width; ++j)
+                v[a_width + j] = bf16_value(b[t * b_row_stride + (int64_t)g * b_width + j]);
+            if (hadamard_n == 128) {
+                hqo_fwht(v, 128);
+                for (int j = 0; j < 128; ++j)
+                    v[j] = v[j] * c;
+            }
+            int64_t grp = t * G + g;
+            float s;
+            quant_group_fp8(v, 128, out + grp * 128, &s, pre ? pre + grp * 128 : 0);
+            if (scale_layout == 0)
+                scales[grp] = s;
+            else
+                scales[(int64_t)g * scale_ld + t] = s;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------ SwiGLU exp */
+/*
+ * exp(x) in binary32, written from the mathematics so that both sides of the
+ * comparison evaluate one fixed sequence of IEEE operations (the pages give
+ * no exp algorithm; [QMOE] only says SiLU/SwiGLU run in FP32):
+ *  - Cody & Waite argument reduction (W. J. Cody, W. Waite, "Software Manual
+ *    for the Elementary Functions", 1980): k = rint(x * log2(e)),
+ *    r = (x - k * LN2_HI) - k * LN2_LO, each step one fmaf;
+ *  - e^r by its Taylor series to degree 7 (|r| <= ln2/2, truncation error
+ *    below 6e-9 relative), Horner form with fmaf;
+ *  - multiply by 2^k, split in two exact power-of-two steps at the ends of
+ *    the exponent range so that only the last multiply rounds.
+ * x > 88.8 -> +inf, x < -104 -> +0 (both beyond binary32 range), NaN -> NaN.
+ */
+static float pow2i(int k) /* 2^k for -126 <= k <= 127 */
+{
+    uint32_t u = (uint32_t)(k + 127) << 23;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+float hqo_exp(float x)
+{
+    if (isnan(x))
+        return x;
+    if (x > 88.8f)
+        return INFINITY;
+    if (x < -104.0f)
+        return 0.0f;
+    const float LOG2E = 1.44269502f;       /* 0x3FB8AA3B */
+    const float LN2_HI = 0.693145752f;     /* 0x3F317200: 15 significant bits */
+    const float LN2_LO = 1.42860677e-06f;  /* 0x35BFBE8E: ln2 - LN2_HI */
+    float k = nearbyintf(x * LOG2E);
+    float r = fmaf(-k, LN2_HI, x);
+    r = fmaf(-k, LN2_LO, r);
+    /* Taylor coefficients 1/n!, each rounded once to binary32, n = 7 .. 0 */
+    float p = 1.0f / 5040.0f;
+    p = fmaf(p, r, 1.0f / 720.0f);
+    p = fmaf(p, r, 1.0f / 120.0f);
+    p = fmaf(p, r, 1.0f / 24.0f);
+    p = fmaf(p, r, 1.0f / 6.0f);
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ki = (int)k;
+    if (ki > 127)
+        return (p * pow2i(127)) * pow2i(ki - 127);
+    if (ki < -126)
+        return (p * pow2i(ki + 100)) * pow2i(-100);
+    return p * pow2i(ki);
+}
+
+void hqo_exp_array(const float *in, float *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = hqo_exp(in[i]);
+}
+
+/* SiLU(g) * u in binary32 [QMOE]: silu = g / (1 + exp(-g)), one IEEE
+ * division; no rounding to a narrower type in between. */
+static float swiglu(float g, float u)
+{
+    float e = hqo_exp(-g);
+    float silu = g / (1.0f + e);
+    return silu * u;
+}
+
+/*
+ * QMoE dynamic FP8 activations [QMOE]: rows of K_out values, quantized in
+ * consecutive groups of 128 with the FP8 rule above.
+ *   mode 0: in is BF16 [M, K_out]
+ *   mode 1: in is FP32 [M, K_out]
+ *   mode 2: in is FP32 [M, 2*K_out]; gate = columns 0..K_out-1, up = columns
+ *           K_out..2*K_out-1 ("2x2048": the reading is two halves, not an
+ *           interleave); the quantized value is SiLU(gate) * up.
+ * out: [M, K_out] codes; scales: [M, K_out/128] row major.
+ */
+int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
+                        uint8_t *out, float *scales, float *pre)
+{
+    if (K_out % 128 != 0 || mode < 0 || mode > 2)
+        return -1;
+    const int64_t groups = K_out / 128;
+    float y[128];
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t g = 0; g < groups; ++g) {
+            for (int j = 0; j < 128; ++j) {
+                int64_t col = g * 128 + j;
+                if (mode == 0)
+                    y[j] = bf16_value(((const uint16_t *)in)[m * K_out + col]);
+                else if (mode == 1)
+                    y[j] = ((const float *)in)[m * K_out + col];
+                else {
+                    const float *row = (const float *)in + m * 2 * K_out;
+                    y[j] = swiglu(row[col], row[K_out + col]);
+                }
+            }
+            int64_t grp = m * groups + g;
+            quant_group_fp8(y, 128, out + grp * 128, &scales[grp], pre ? pre + grp * 128 : 0);
+        }
+    return 0;
+}
+
+/* ----------------------------------------------------------------- NVFP4 */
+/*
+ * NVFP4 two-level scaling.  The pages name the format ("NVFP4", E2M1 codes
+ * with E4M3 1x16 block scales and an FP32 global scale) but print no formula.
+ * Reading, per section and per direction:
+ *   A     = max |v| over the section's values
+ *   S_enc = 2688 / A   (6 * 448: the section's amax maps to the largest
+ *                       E2M1 value times the largest E4M3 value); 1 if A == 0
+ *                       or the quotient is not finite
+ *   sdec  = 1 / S_enc
+ * and per block of 16 values:
+ *   a_b   = max |v_i|
+ *   sf    = e4m3((a_b / 6) * S_enc)
+ *   enc   = sf == 0 ? 0 : S_enc / float(sf)
+ *   code  = e2m1(v_i * enc)
+ * so that v_i ~= e2m1_value(code) * float(sf) * sdec.
+ */
+static float global_encode_scale(float A)
+{
+    float S = 2688.0f / A;
+    if (A == 0.0f || !isfinite(S))
+        S = 1.0f;
+    return S;
+}
+
+/* Quantize one block of 16 values; codes packed two per byte, element 2k in
+ * the low nibble and 2k+1 in the high nibble (reading: the pages are silent
+ * on the packing). */
+static void nvfp4_block(const float *v, float S_enc, uint8_t *codes8, uint8_t *sf_out, float *pre)
+{
+    float ab = 0.0f;
+    for (int i = 0; i < 16; ++i)
+        ab = fmaxf(ab, fabsf(v[i]));
+    uint8_t sf = hqo_e4m3_encode((ab / 6.0f) * S_enc);
+    float sff = hqo_e4m3_decode(sf);
+    float enc = sff == 0.0f ? 0.0f : S_enc / sff;
+    for (int k = 0; k < 8; ++k) {
+        float t0 = v[2 * k] * enc, t1 = v[2 * k + 1] * enc;
+        if (pre) {
+            pre[2 * k] = t0;
+            pre[2 * k + 1] = t1;
+        }
+        codes8[k] = (uint8_t)((hqo_e2m1_encode(t0) & 0xF) | ((hqo_e2m1_encode(t1) & 0xF) << 4));
+    }
+    *sf_out = sf;
+}
+
+/* The 16-point random Hadamard transform of [GRP]/[FUS]: v = 0.25 * H16 *
+ * diag(sigma) * x, sigma_i = -1 where bit i of sign_mask is set (i is the
+ * position inside the block). */
+static void rht16(const float *x, uint16_t sign_mask, float *v)
+{
+    for (int i = 0; i < 16; ++i)
+        v[i] = ((sign_mask >> i) & 1) ? -x[i] : x[i];
+    hqo_fwht(v, 16);
+    for (int i = 0; i < 16; ++i)
+        v[i] = v[i] * 0.25f;
+}
+
+/*
+ * Grouped RHT + NVFP4 cast [GRP], [FUS].  x: BF16 [M, K] row major, rows split
+ * into S consecutive sections of split_rows[s] rows (each a multiple of 128,
+ * [FUS]'s fusion rule; K a multiple of 128).
+ * flags bit 0 (rowwise): plain cast of x along K (the pages' rowwise output
+ *   carries no RHT):  row_codes [M, K/2], row_sf [M, K/16].
+ * flags bit 1 (columnwise): per section, the 16-point RHT along M (16
+ *   consecutive rows of one column), cast, stored transposed: section s
+ *   starting at row r0 owns col_codes[K*r0/2 ...] as [K, M_s/2] and
+ *   col_sf[K*r0/16 ...] as [K, M_s/16].
+ * amax_*[s], sdec_*[s] receive A and 1/S_enc of the requested directions;
+ * an empty section gives A = 0, sdec = 1.  row_pre / col_pre, when given,
+ * receive the value rounded to E2M1 per element, in the output's layout.
+ */
+int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
+                        const int64_t *split_rows, int S, uint16_t sign_mask, unsigned flags,
+                        uint8_t *row_codes, uint8_t *row_sf, uint8_t *col_codes, uint8_t *col_sf,
+                        float *amax_row, float *amax_col, float *sdec_row, float *sdec_col,
+                        float *row_pre, float *col_pre)
+{
+    if (K % 128 != 0 || S < 0)
+        return -1;
+    int64_t total = 0;
+    for (int s = 0; s < S; ++s) {
+        if (split_rows[s] < 0 || split_rows[s] % 128 != 0)
+            return -1;
+        total += split_rows[s];
+    }
+    if (total != M)
+        return -1;
+
+    int64_t r0 = 0;
+    float blk[16], v[16];
+    for (int s = 0; s < S; ++s) {
+        const int64_t Ms = split_rows[s];
+        if (flags & 1) {
+            float A = 0.0f;
+            for (int64_t r = r0; r < r0 + Ms; ++r)
+                for (int64_t k = 0; k < K; ++k)
+                    A = fmaxf(A, fabsf(bf16_value(x[r * K + k])));
+            float S_enc = global_encode_scale(A);
+            amax_row[s] = A;
+            sdec_row[s] = 1.0f / S_enc;
+            for (int64_t r = r0; r < r0 + Ms; ++r)
+                for (int64_t kb = 0; kb < K / 16; ++kb) {
+                    for (int i = 0; i < 16; ++i)
+                        blk[i] = bf16_value(x[r * K + kb * 16 + i]);
+                    nvfp4_block(blk, S_enc, row_codes + r * (K / 2) + kb * 8,
+                                row_sf + r * (K / 16) + kb,
+                                row_pre ? row_pre + r * K + kb * 16 : 0);
+                }
+        }
+        if (flags & 2) {
+            /* first pass: section amax of the rotated values */
+            float A = 0.0f;
+            for (int64_t c = 0; c < K; ++c)
+                for (int64_t mb = 0; mb < Ms / 16; ++mb) {
+                    for (int i = 0; i < 16; ++i)
+                        blk[i] = bf16_value(x[(r0 + mb * 16 + i) * K + c]);
+                    rht16(blk, sign_mask, v);
+                    for (int i = 0; i < 16; ++i)
+                        A = fmaxf(A, fabsf(v[i]));
+                }
+            float S_enc = global_encode_scale(A);
+            amax_col[s] = A;
+            sdec_col[s] = 1.0f / S_enc;
+            uint8_t *cc = col_codes + K * r0 / 2;
+            uint8_t *cs = col_sf + K * r0 / 16;
+            /* second pass: cast, transposed [K, Ms] */
+            for (int64_t c = 0; c < K; ++c)
+                for (int64_t mb = 0; mb < Ms / 16; ++mb) {
+                    for (int i = 0; i < 16; ++i)
+                        blk[i] = bf16_value(x[(r0 + mb * 16 + i) * K + c]);
+                    rht16(blk, sign_mask, v);
+                    nvfp4_block(v, S_enc, cc + c * (Ms / 2) + mb * 8, cs + c * (Ms / 16) + mb,
+                                col_pre ? col_pre + K * r0 + c * Ms + mb * 16 : 0);
+                }
+        }
+        if (Ms == 0) {
+            if (flags & 1) { amax_row[s] = 0.0f; sdec_row[s] = 1.0f; }
+            if (flags & 2) { amax_col[s] = 0.0f; sdec_col[s] = 1.0f; }
+        }
+        r0 += Ms;
+    }
+    return 0;
+}
