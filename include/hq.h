@@ -1,0 +1,215 @@
+/*
+ * hq.h -- C ABI of the hq library: Hadamard rotation fused with block-scaled
+ * low-precision quantization (NVFP4 and FP8 E4M3) on NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every call below:
+ *  - Pointers are CUDA device pointers owned by the caller, unless a comment
+ *    says "host".  The library allocates no memory, never synchronizes the
+ *    stream (hq_get_error excepted) and reads no environment variables.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default).
+ *  - Every argument is checked before anything is launched; a violation
+ *    returns a nonzero hq_status and leaves all outputs untouched.  There is no
+ *    fallback path: an unsupported request is an error.
+ *  - Calls are asynchronous: a status of HQ_OK means the work was enqueued.
+ *  - BF16 tensors are passed as their 16-bit patterns, FP8 E4M3 codes as
+ *    bytes, NVFP4 E2M1 codes two per byte (element 2k in the low nibble).
+ *
+ * Sources for the operations (page titles):
+ *  [GRP] TransformerEngine PR #2564 "[NVFP4][MOE] Bug Fix for NVFP4 Grouped
+ *        Quant": the grouped row-cast / column-Hadamard-transform-cast kernel
+ *        over MoE split sections, and its caller-provided 4-byte tile
+ *        scheduler workspace (replacing a per-call cudaMallocAsync), plus the
+ *        reviewers' request for a workspace-size query.
+ *  [FUS] TransformerEngine PR #2555 review comments: split_section % 128
+ *        fusion rule, rht_matrix, rowwise-only output needs no RHT, the RHT'd
+ *        columnwise output is the transposed [cols, rows] tensor.
+ *  [DSA] TensorRT-LLM PR #15158 "[#13061][bugfix] Add rotate_activation to DSA
+ *        fused_cat_fp8 path": cat([pe, nope]) -> Hadamard rotation ->
+ *        fp8_quantize_1x128, scales transposed.
+ *  [QMOE] onnxruntime PR #33644 (QMoE activation_quantization="dynamic_fp8"),
+ *        Description: K128 groups, saturating nearest-even E4M3,
+ *        max(amax, 1e-10) * float32(1/448) scales, FP32 SiLU/SwiGLU before
+ *        the second quantizer, explicit errors instead of fallbacks.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hq_status {
+    HQ_OK = 0,
+    HQ_ERR_NULL = 1,        /* a required pointer is NULL */
+    HQ_ERR_SHAPE = 2,       /* sizes negative, inconsistent or too large */
+    HQ_ERR_ALIGN = 3,       /* pointer/stride not 16-byte aligned, or a size
+                               not a multiple of the required block */
+    HQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the query */
+    HQ_ERR_UNSUPPORTED = 5, /* unknown flag, mode, layout or transform size */
+    HQ_ERR_CUDA = 6,        /* the CUDA runtime reported an error */
+    HQ_ERR_TIMEOUT = 7      /* a bounded device-side wait gave up */
+} hq_status;
+
+/* hq_group_rht_quant flags */
+#define HQ_ROWWISE 1u      /* rowwise NVFP4 output (plain cast along K) */
+#define HQ_COLWISE 2u      /* columnwise NVFP4 output (RHT16 along M, transposed) */
+#define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
+                              instead of one launch in which each section's
+                              cast follows its amax while the rows are still
+                              in L2; results are identical */
+
+/* hq_cat_rotate_fp8 scale layouts */
+#define HQ_SCALE_ROWMAJOR 0   /* scale of group (t, g) at scales[t * G + g] */
+#define HQ_SCALE_TRANSPOSED 1 /* scale of group (t, g) at scales[g * scale_ld + t] */
+
+/* hq_swiglu_fp8_k128 modes */
+#define HQ_ACT_NONE_BF16 0  /* in: BF16 [M, K_out] */
+#define HQ_ACT_NONE_F32 1   /* in: FP32 [M, K_out] */
+#define HQ_ACT_SWIGLU_F32 2 /* in: FP32 [M, 2*K_out], gate = cols [0, K_out),
+                               up = cols [K_out, 2*K_out); value SiLU(gate)*up */
+
+/* hq_convert formats */
+#define HQ_FMT_E4M3 0 /* one E4M3 code per output byte */
+#define HQ_FMT_E2M1 1 /* one E2M1 code per output byte (low nibble) */
+
+#define HQ_MAX_SECTIONS 256
+
+/* Library version, (major << 16) | minor. */
+int hq_version(void);
+
+/* Static description of a status code. */
+const char *hq_status_string(hq_status s);
+
+/*
+ * Workspace bytes hq_group_rht_quant needs for `num_sections` sections
+ * (1 <= num_sections <= HQ_MAX_SECTIONS; 0 otherwise).  The first 4 bytes
+ * are the tile-scheduler counter of [GRP]; per-section amax accumulators,
+ * completion counters and an error word follow.  The size query is the
+ * reviewers' proposal in [GRP].
+ */
+size_t hq_group_rht_quant_workspace_size(int num_sections);
+
+/*
+ * Put a workspace into its rest state (all zero).  Call once after
+ * allocating it (an enqueued memset on `stream`).  Every hq_group_rht_quant
+ * call leaves the workspace in the rest state again, so no per-call memset
+ * is needed.  Two calls that share one workspace must not overlap in time
+ * (same stream, or ordered by events).
+ * Errors: HQ_ERR_NULL, HQ_ERR_ALIGN (ws not 16-byte aligned), HQ_ERR_CUDA.
+ */
+hq_status hq_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Read and clear the workspace's device error word.  Synchronizes `stream`.
+ * *err_out (host) receives 0, or HQ_ERR_TIMEOUT if a bounded device wait of
+ * an earlier call gave up (that call's outputs are then incomplete).
+ */
+hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *stream);
+
+/*
+ * Grouped random-Hadamard-transform + NVFP4 cast over MoE split sections
+ * [GRP], [FUS].
+ *
+ *  x          BF16 [M, K] row major.  16-byte aligned.
+ *  M, K       rows, columns.  K > 0 and K % 128 == 0.
+ *  split_rows HOST int64 [S]: rows per section, each >= 0 and a multiple of
+ *             128 ([FUS] fusion rule), summing to M.  Empty sections allowed.
+ *  S          number of sections, 1 <= S <= HQ_MAX_SECTIONS.
+ *  sign_mask  the random sign vector of the 16-point RHT: bit i set means
+ *             sigma_i = -1 for position i of each 16-row block.
+ *  flags      HQ_ROWWISE | HQ_COLWISE (at least one), optionally HQ_TWO_PASS.
+ *
+ * For section s (rows [r0, r0 + M_s)) and each requested direction:
+ *   A_s = max |v| over the section's values (v = x rowwise; v = RHT16 output
+ *   columnwise), S_enc = 2688 / A_s (1 when A_s == 0 or not finite),
+ *   sdec = 1 / S_enc; for each block of 16 values along the quantized
+ *   direction: sf = E4M3((a_b / 6) * S_enc), code_i = E2M1(v_i * S_enc / sf)
+ *   (0 when sf == 0); saturating round-to-nearest-even conversions.
+ *   RHT16 of a block: v = 0.25 * H16 * diag(sigma) * x, H16 the Sylvester
+ *   Hadamard matrix.
+ *
+ * Outputs (device; each 16-byte aligned; amax/sdec 4-byte aligned):
+ *  row_codes  uint8 [M, K/2]     rowwise E2M1 codes          (HQ_ROWWISE)
+ *  row_sf     uint8 [M, K/16]    rowwise E4M3 block scales   (HQ_ROWWISE)
+ *  col_codes  uint8 [M*K/2]      per section s: [K, M_s/2] at byte K*r0/2
+ *  col_sf     uint8 [M*K/16]     per section s: [K, M_s/16] at byte K*r0/16
+ *  amax_row, sdec_row  float [S] (HQ_ROWWISE)
+ *  amax_col, sdec_col  float [S] (HQ_COLWISE)
+ *  Pointers of a direction not requested may be NULL.
+ *
+ *  ws, ws_bytes  caller workspace, >= hq_group_rht_quant_workspace_size(S),
+ *                16-byte aligned, in the rest state (hq_workspace_init).
+ * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE,
+ *         HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
+ * Inputs must be finite (NaN/inf are outside the NVFP4 contract).
+ */
+hq_status hq_group_rht_quant(const void *x, int64_t M, int64_t K,
+                             const int64_t *split_rows, int S, uint16_t sign_mask,
+                             unsigned flags,
+                             uint8_t *row_codes, uint8_t *row_sf,
+                             uint8_t *col_codes, uint8_t *col_sf,
+                             float *amax_row, float *amax_col,
+                             float *sdec_row, float *sdec_col,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Concatenate -> 128-point Hadamard rotation -> FP8 E4M3 1x128 quantization
+ * [DSA] (the DSA indexer's q/k preparation), with the scale rule of [QMOE].
+ *
+ *  a          BF16; element j of group g of row t is
+ *             a[t * a_row_stride + g * a_width + j], 0 <= j < a_width.
+ *  b          BF16 or NULL (when b_width == 0); same indexing with b_*.
+ *             The 128-vector of (t, g) is a-part followed by b-part
+ *             ([pe, nope]); a_width + b_width == 128, both multiples of 8.
+ *  M, G       rows (tokens) and groups (heads) per row.
+ *  hadamard_n 128 (rotate by H128 / sqrt(128), Sylvester order) or 0 (none).
+ *  out_fp8    uint8 [M, G*128] codes: (t, g, j) at (t * G + g) * 128 + j.
+ *  scales     float: group scale s = max(amax, 1e-10) * float32(1/448),
+ *             codes = E4M3(y / s) (IEEE division, saturating RNE).
+ *             scale_layout HQ_SCALE_ROWMAJOR: [M, G] (scale_ld ignored);
+ *             HQ_SCALE_TRANSPOSED: [G, scale_ld], scale_ld >= M.
+ *  ws, ws_bytes  unused (the call needs no workspace; may be NULL / 0).
+ * Alignment: a, b, out 16 bytes; strides multiples of 8 elements.
+ * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
+ *         HQ_ERR_CUDA.
+ */
+hq_status hq_cat_rotate_fp8(const void *a, int64_t a_row_stride, int a_width,
+                            const void *b, int64_t b_row_stride, int b_width,
+                            int64_t M, int G, int hadamard_n,
+                            uint8_t *out_fp8, float *scales, int scale_layout,
+                            int64_t scale_ld, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * QMoE dynamic FP8 activation quantizer [QMOE]: each row of K_out values is
+ * split into consecutive groups of 128; each group gets the FP8 rule above.
+ *  mode     HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32 or HQ_ACT_SWIGLU_F32 (the value
+ *           quantized is SiLU(gate) * up computed in FP32, SiLU(g) =
+ *           g / (1 + exp(-g)), with no narrower rounding in between).
+ *  in       see the modes; row stride K_out (or 2*K_out for SwiGLU).
+ *  out_fp8  uint8 [M, K_out];  scales float [M, K_out/128] row major.
+ *  K_out    multiple of 128.   ws, ws_bytes unused (may be NULL / 0).
+ * Alignment: in and out 16 bytes, scales 4 bytes.
+ * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
+ *         HQ_ERR_CUDA.
+ */
+hq_status hq_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
+                             uint8_t *out_fp8, float *scales,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Element-wise conversion of FP32 values with the library's own device
+ * conversion routines (the ones every kernel above uses): E4M3 (saturating,
+ * nearest even) or E2M1 (one nibble per byte).  n >= 0; in and out may have
+ * any alignment.
+ * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA.
+ */
+hq_status hq_convert(int fmt, const float *in, uint8_t *out, int64_t n, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H */

@@ -1,0 +1,213 @@
+"""Python binding of the hq C ABI (include/hq.h): argument marshalling only.
+
+Every function below passes raw device pointers and sizes to the compiled
+library ``libhq.so`` (CUDA kernels for sm_100a); no step of the computation
+runs in Python or PyTorch.  PyTorch is used for device memory and streams.
+If the library is missing or fails to load, importing the compute functions
+raises: there is no fallback.
+
+Low-level calls (``hq_*``) take caller-allocated output tensors exactly like
+the C functions.  ``group_rht_quant``, ``cat_rotate_fp8`` and
+``swiglu_fp8_k128`` allocate the outputs with torch and call them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhq.so")
+
+HQ_OK, HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA, \
+    HQ_ERR_TIMEOUT = range(8)
+HQ_ROWWISE, HQ_COLWISE, HQ_TWO_PASS = 1, 2, 8
+HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
+HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
+HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1
+HQ_MAX_SECTIONS = 256
+
+EXPORTED = (
+    "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
+    "hq_get_error", "hq_group_rht_quant", "hq_cat_rotate_fp8", "hq_swiglu_fp8_k128", "hq_convert",
+)
+
+
+class HQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libhq.so (raises OSError if it is missing: build it first)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} not found: run nvfp4_quantization_group_b200/_build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, sz, u = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint
+        c_int = ctypes.c_int
+        L.hq_version.restype = c_int
+        L.hq_version.argtypes = []
+        L.hq_status_string.restype = ctypes.c_char_p
+        L.hq_status_string.argtypes = [c_int]
+        L.hq_group_rht_quant_workspace_size.restype = sz
+        L.hq_group_rht_quant_workspace_size.argtypes = [c_int]
+        L.hq_workspace_init.restype = c_int
+        L.hq_workspace_init.argtypes = [P, sz, P]
+        L.hq_get_error.restype = c_int
+        L.hq_get_error.argtypes = [P, sz, ctypes.POINTER(ctypes.c_uint32), P]
+        L.hq_group_rht_quant.restype = c_int
+        L.hq_group_rht_quant.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
+                                         P, P, P, P, P, P, P, P, P, sz, P]
+        L.hq_cat_rotate_fp8.restype = c_int
+        L.hq_cat_rotate_fp8.argtypes = [P, i64, c_int, P, i64, c_int, i64, c_int, c_int,
+                                        P, P, c_int, i64, P, sz, P]
+        L.hq_swiglu_fp8_k128.restype = c_int
+        L.hq_swiglu_fp8_k128.argtypes = [c_int, P, i64, i64, P, P, P, sz, P]
+        L.hq_convert.restype = c_int
+        L.hq_convert.argtypes = [c_int, P, P, i64, P]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().hq_status_string(int(status)).decode()
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != HQ_OK:
+        raise HQError(status, what)
+
+
+# ------------------------------------------------------------- C ABI calls
+def hq_version() -> int:
+    return lib().hq_version()
+
+
+def hq_group_rht_quant_workspace_size(num_sections: int) -> int:
+    return int(lib().hq_group_rht_quant_workspace_size(int(num_sections)))
+
+
+def hq_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(lib().hq_workspace_init(_p(ws), ws.numel() * ws.element_size(), _stream(stream)), "hq_workspace_init")
+
+
+def hq_get_error(ws: torch.Tensor, stream=None) -> int:
+    err = ctypes.c_uint32(0)
+    _check(lib().hq_get_error(_p(ws), ws.numel() * ws.element_size(), ctypes.byref(err), _stream(stream)),
+           "hq_get_error")
+    return int(err.value)
+
+
+def hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, row_codes, row_sf, col_codes, col_sf,
+                       amax_row, amax_col, sdec_row, sdec_col, ws, stream=None) -> None:
+    splits = (ctypes.c_int64 * len(split_rows))(*[int(v) for v in split_rows])
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().hq_group_rht_quant(_p(x), int(M), int(K), ctypes.cast(splits, ctypes.c_void_p), int(S),
+                                    int(sign_mask) & 0xFFFF, int(flags), _p(row_codes), _p(row_sf),
+                                    _p(col_codes), _p(col_sf), _p(amax_row), _p(amax_col), _p(sdec_row),
+                                    _p(sdec_col), _p(ws), ws_bytes, _stream(stream)), "hq_group_rht_quant")
+
+
+def hq_cat_rotate_fp8(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, out_fp8, scales,
+                      scale_layout, scale_ld, stream=None) -> None:
+    _check(lib().hq_cat_rotate_fp8(_p(a), int(a_row_stride), int(a_width), _p(b), int(b_row_stride),
+                                   int(b_width), int(M), int(G), int(hadamard_n), _p(out_fp8), _p(scales),
+                                   int(scale_layout), int(scale_ld), None, 0, _stream(stream)),
+           "hq_cat_rotate_fp8")
+
+
+def hq_swiglu_fp8_k128(mode, inp, M, K_out, out_fp8, scales, stream=None) -> None:
+    _check(lib().hq_swiglu_fp8_k128(int(mode), _p(inp), int(M), int(K_out), _p(out_fp8), _p(scales), None, 0,
+                                    _stream(stream)), "hq_swiglu_fp8_k128")
+
+
+def hq_convert(fmt, inp, out, n, stream=None) -> None:
+    _check(lib().hq_convert(int(fmt), _p(inp), _p(out), int(n), _stream(stream)), "hq_convert")
+
+
+# ------------------------------------------------- allocating conveniences
+def new_workspace(num_sections: int, device="cuda", stream=None) -> torch.Tensor:
+    """A workspace for `num_sections` sections, put into its rest state once."""
+    nbytes = hq_group_rht_quant_workspace_size(num_sections)
+    if nbytes == 0:
+        raise HQError(HQ_ERR_SHAPE, "new_workspace")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    hq_workspace_init(ws, stream)
+    return ws
+
+
+def group_outputs(M: int, K: int, S: int, flags: int = HQ_ROWWISE | HQ_COLWISE, device="cuda") -> dict:
+    u8 = dict(dtype=torch.uint8, device=device)
+    f32 = dict(dtype=torch.float32, device=device)
+    out = {}
+    if flags & HQ_ROWWISE:
+        out.update(row_codes=torch.empty((M, K // 2), **u8), row_sf=torch.empty((M, K // 16), **u8),
+                   amax_row=torch.empty(S, **f32), sdec_row=torch.empty(S, **f32))
+    if flags & HQ_COLWISE:
+        out.update(col_codes=torch.empty(M * K // 2, **u8), col_sf=torch.empty(M * K // 16, **u8),
+                   amax_col=torch.empty(S, **f32), sdec_col=torch.empty(S, **f32))
+    return out
+
+
+def group_rht_quant(x: torch.Tensor, split_rows, sign_mask: int, flags: int = HQ_ROWWISE | HQ_COLWISE,
+                    ws: torch.Tensor | None = None, out: dict | None = None, stream=None) -> dict:
+    """Grouped RHT16 + NVFP4 cast of a BF16 [M, K] CUDA tensor (see hq.h)."""
+    M, K = x.shape
+    S = len(split_rows)
+    if ws is None:
+        ws = new_workspace(S, x.device, stream)
+    if out is None:
+        out = group_outputs(M, K, S, flags, x.device)
+    g = out.get
+    hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, g("row_codes"), g("row_sf"), g("col_codes"),
+                       g("col_sf"), g("amax_row"), g("amax_col"), g("sdec_row"), g("sdec_col"), ws, stream)
+    return out
+
+
+def cat_rotate_fp8(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 128,
+                   scale_layout: int = HQ_SCALE_ROWMAJOR, scale_ld: int | None = None, stream=None):
+    """a: BF16 [M, G, a_width], b: BF16 [M, G, b_width] or None -> (codes [M, G*128], scales)."""
+    M, G, aw = a.shape
+    bw = 0 if b is None else b.shape[-1]
+    codes = torch.empty((M, G * 128), dtype=torch.uint8, device=a.device)
+    if scale_layout == HQ_SCALE_ROWMAJOR:
+        scales = torch.empty((M, G), dtype=torch.float32, device=a.device)
+        ld = G
+    else:
+        ld = M if scale_ld is None else scale_ld
+        scales = torch.empty((G, ld), dtype=torch.float32, device=a.device)
+    hq_cat_rotate_fp8(a, a.stride(0), aw, b, 0 if b is None else b.stride(0), bw, M, G, hadamard_n, codes,
+                      scales, scale_layout, ld, stream)
+    return codes, scales
+
+
+def swiglu_fp8_k128(mode: int, inp: torch.Tensor, K_out: int, stream=None):
+    """K128 FP8 quantization (modes HQ_ACT_*) -> (codes [M, K_out], scales [M, K_out/128])."""
+    M = inp.shape[0]
+    codes = torch.empty((M, K_out), dtype=torch.uint8, device=inp.device)
+    scales = torch.empty((M, K_out // 128), dtype=torch.float32, device=inp.device)
+    hq_swiglu_fp8_k128(mode, inp, M, K_out, codes, scales, stream)
+    return codes, scales

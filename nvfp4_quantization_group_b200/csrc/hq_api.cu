@@ -1,0 +1,275 @@
+// hq_api.cu -- the extern "C" entry points of include/hq.h: argument checks,
+// kernel parameter blocks, grid sizing and launches.  No allocation, no
+// synchronization (hq_get_error excepted), no environment reads.
+#include <string.h>
+
+#include <mutex>
+
+#include "hq_internal.h"
+
+using namespace hq;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sms = 0;
+    int nv_blocks_per_sm = 0;
+    int cat_blocks_per_sm = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+// SM count and resident CTAs per SM of the persistent kernels, per device.
+const DeviceInfo* device_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_dev_once[dev], [dev] {
+        DeviceInfo d;
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        d.nv_blocks_per_sm = nvfp4_blocks_per_sm();
+        d.cat_blocks_per_sm = cat_rotate_blocks_per_sm();
+        g_dev[dev] = d;
+    });
+    const DeviceInfo* d = &g_dev[dev];
+    return d->sms > 0 ? d : nullptr;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+inline hq_status launch_status() {
+    return cudaPeekAtLastError() == cudaSuccess ? HQ_OK : (cudaGetLastError(), HQ_ERR_CUDA);
+}
+
+size_t nv_ws_words(int S) { return (size_t)NV_WS_HEADER + 3 * (size_t)S; }
+
+}  // namespace
+
+extern "C" {
+
+int hq_version(void) { return (0 << 16) | 1; }
+
+const char* hq_status_string(hq_status s) {
+    switch (s) {
+        case HQ_OK: return "ok";
+        case HQ_ERR_NULL: return "required pointer is NULL";
+        case HQ_ERR_SHAPE: return "sizes negative, inconsistent or too large";
+        case HQ_ERR_ALIGN: return "misaligned pointer/stride or size not a multiple of the block";
+        case HQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case HQ_ERR_UNSUPPORTED: return "unsupported flag, mode, layout or transform size";
+        case HQ_ERR_CUDA: return "CUDA runtime error";
+        case HQ_ERR_TIMEOUT: return "bounded device wait gave up";
+    }
+    return "unknown status";
+}
+
+size_t hq_group_rht_quant_workspace_size(int num_sections) {
+    if (num_sections < 1 || num_sections > HQ_MAX_SECTIONS) return 0;
+    const size_t bytes = nv_ws_words(num_sections) * sizeof(uint32_t);
+    return (bytes + 255) & ~(size_t)255;
+}
+
+hq_status hq_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws) return HQ_ERR_NULL;
+    if (!aligned16(ws)) return HQ_ERR_ALIGN;
+    if (cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) != cudaSuccess) return HQ_ERR_CUDA;
+    return HQ_OK;
+}
+
+hq_status hq_get_error(void* ws, size_t ws_bytes, uint32_t* err_out, void* stream) {
+    if (!ws || !err_out) return HQ_ERR_NULL;
+    if (ws_bytes < NV_WS_HEADER * sizeof(uint32_t)) return HQ_ERR_WORKSPACE;
+    uint32_t* err = static_cast<uint32_t*>(ws) + 2;
+    uint32_t host = 0;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&host, err, sizeof host, cudaMemcpyDeviceToHost, st) != cudaSuccess) return HQ_ERR_CUDA;
+    if (cudaMemsetAsync(err, 0, sizeof(uint32_t), st) != cudaSuccess) return HQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HQ_ERR_CUDA;
+    *err_out = host;
+    return HQ_OK;
+}
+
+hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
+                             uint16_t sign_mask, unsigned flags, uint8_t* row_codes, uint8_t* row_sf,
+                             uint8_t* col_codes, uint8_t* col_sf, float* amax_row, float* amax_col,
+                             float* sdec_row, float* sdec_col, void* ws, size_t ws_bytes, void* stream) {
+    // ---- argument checks (nothing is launched on failure)
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
+    const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
+    if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
+    if (!split_rows || !ws) return HQ_ERR_NULL;
+    if (do_row && (!row_codes || !row_sf || !amax_row || !sdec_row)) return HQ_ERR_NULL;
+    if (do_col && (!col_codes || !col_sf || !amax_col || !sdec_col)) return HQ_ERR_NULL;
+    if (S < 1 || S > HQ_MAX_SECTIONS || M < 0 || K <= 0) return HQ_ERR_SHAPE;
+    if (M > 0 && !x) return HQ_ERR_NULL;
+    if (K % NV_TILE != 0) return HQ_ERR_ALIGN;
+    if (M * K >= ((int64_t)1 << 40) || M >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
+    int64_t total = 0;
+    for (int s = 0; s < S; ++s) {
+        if (split_rows[s] < 0) return HQ_ERR_SHAPE;
+        if (split_rows[s] % NV_TILE != 0) return HQ_ERR_ALIGN;
+        total += split_rows[s];
+    }
+    if (total != M) return HQ_ERR_SHAPE;
+    if ((M > 0 && !aligned16(x)) || !aligned16(ws)) return HQ_ERR_ALIGN;
+    if (do_row && (!aligned16(row_codes) || !aligned16(row_sf) || !aligned4(amax_row) || !aligned4(sdec_row)))
+        return HQ_ERR_ALIGN;
+    if (do_col && (!aligned16(col_codes) || !aligned16(col_sf) || !aligned4(amax_col) || !aligned4(sdec_col)))
+        return HQ_ERR_ALIGN;
+    if (ws_bytes < hq_group_rht_quant_workspace_size(S)) return HQ_ERR_WORKSPACE;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return HQ_ERR_CUDA;
+
+    // ---- schedule: per non-empty section an amax segment and a cast segment
+    NvParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint16_t*>(x);
+    p.K = K;
+    p.row_codes = row_codes; p.row_sf = row_sf; p.col_codes = col_codes; p.col_sf = col_sf;
+    p.amax_row = amax_row; p.amax_col = amax_col; p.sdec_row = sdec_row; p.sdec_col = sdec_col;
+    p.ws = static_cast<uint32_t*>(ws);
+    p.S = S;
+    p.sign_mask = sign_mask;
+    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE);
+    p.col_tiles = (int)(K / NV_TILE);
+    int row0 = 0;
+    int live[HQ_MAX_SECTIONS];
+    int nlive = 0;
+    for (int s = 0; s < S; ++s) {
+        p.sec_row0[s] = row0;
+        row0 += (int)split_rows[s];
+        if (split_rows[s] > 0) live[nlive++] = s;
+    }
+    p.sec_row0[S] = row0;
+
+    auto tiles_of = [&](int s) { return (uint32_t)(split_rows[s] / NV_TILE) * (uint32_t)p.col_tiles; };
+    auto add_seg = [&](NvParams& q, int s, int phase, uint32_t& next) {
+        q.seg_start[q.nseg] = next;
+        q.seg_info[q.nseg] = (uint16_t)(s | (phase << 15));
+        ++q.nseg;
+        next += tiles_of(s);
+    };
+    cudaStream_t st = (cudaStream_t)stream;
+    const int max_grid = dev->sms * (dev->nv_blocks_per_sm > 0 ? dev->nv_blocks_per_sm : 1);
+    auto launch = [&](NvParams& q, uint32_t items) -> hq_status {
+        q.seg_start[q.nseg] = items;
+        q.total_items = items;
+        const int grid = (int)(items < (uint32_t)max_grid ? (items > 0 ? items : 1) : (uint32_t)max_grid);
+        launch_nvfp4(q, grid, st);
+        return launch_status();
+    };
+
+    if (!(flags & HQ_TWO_PASS)) {
+        // A(s0) A(s1) C(s0) A(s2) C(s1) ... C(s_last)
+        uint32_t next = 0;
+        for (int k = 0; k < nlive; ++k) {
+            add_seg(p, live[k], 0, next);
+            if (k >= 1) add_seg(p, live[k - 1], 1, next);
+        }
+        if (nlive > 0) add_seg(p, live[nlive - 1], 1, next);
+        p.finalize = 1;
+        p.reset_counter = 1;
+        return launch(p, next);
+    }
+    // two launches: all amax tiles, then all cast tiles
+    NvParams pa = p, pc = p;
+    uint32_t na = 0, nc = 0;
+    for (int k = 0; k < nlive; ++k) {
+        add_seg(pa, live[k], 0, na);
+        add_seg(pc, live[k], 1, nc);
+    }
+    pa.finalize = 0;
+    pa.reset_counter = 1;
+    pc.finalize = 1;
+    pc.reset_counter = 1;
+    hq_status r = launch(pa, na);
+    if (r != HQ_OK) return r;
+    return launch(pc, nc);
+}
+
+hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, const void* b,
+                            int64_t b_row_stride, int b_width, int64_t M, int G, int hadamard_n,
+                            uint8_t* out_fp8, float* scales, int scale_layout, int64_t scale_ld,
+                            void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (hadamard_n != 0 && hadamard_n != 128) return HQ_ERR_UNSUPPORTED;
+    if (scale_layout != HQ_SCALE_ROWMAJOR && scale_layout != HQ_SCALE_TRANSPOSED) return HQ_ERR_UNSUPPORTED;
+    if (M < 0 || G <= 0 || a_width < 0 || b_width < 0 || a_width + b_width != 128) return HQ_ERR_SHAPE;
+    if (M == 0) return HQ_OK;
+    if (!a || !out_fp8 || !scales || (b_width > 0 && !b)) return HQ_ERR_NULL;
+    if (a_width % 8 || b_width % 8 || a_row_stride % 8 || b_row_stride % 8) return HQ_ERR_ALIGN;
+    if (a_row_stride < (int64_t)G * a_width || (b_width > 0 && b_row_stride < (int64_t)G * b_width))
+        return HQ_ERR_SHAPE;
+    if (scale_layout == HQ_SCALE_TRANSPOSED && scale_ld < M) return HQ_ERR_SHAPE;
+    if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out_fp8) || !aligned4(scales))
+        return HQ_ERR_ALIGN;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return HQ_ERR_CUDA;
+
+    CatRotateParams p;
+    p.a = static_cast<const uint16_t*>(a);
+    p.b = static_cast<const uint16_t*>(b);
+    p.a_row_stride = a_row_stride;
+    p.b_row_stride = b_row_stride;
+    p.a_width = a_width;
+    p.b_width = b_width;
+    p.nvec = M * G;
+    p.G = G;
+    p.rotate = hadamard_n == 128;
+    p.out = out_fp8;
+    p.scales = scales;
+    p.scale_layout = scale_layout;
+    p.scale_ld = scale_ld;
+    const int64_t tiles = (p.nvec + 127) / 128;
+    const int64_t cap = (int64_t)dev->sms * (dev->cat_blocks_per_sm > 0 ? dev->cat_blocks_per_sm : 1);
+    const int grid = (int)(tiles < cap ? tiles : cap);
+    launch_cat_rotate(p, grid, (cudaStream_t)stream);
+    return launch_status();
+}
+
+hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out, uint8_t* out_fp8,
+                             float* scales, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (mode != HQ_ACT_NONE_BF16 && mode != HQ_ACT_NONE_F32 && mode != HQ_ACT_SWIGLU_F32) return HQ_ERR_UNSUPPORTED;
+    if (M < 0 || K_out <= 0) return HQ_ERR_SHAPE;
+    if (K_out % 128) return HQ_ERR_ALIGN;
+    if (M == 0) return HQ_OK;
+    if (!in || !out_fp8 || !scales) return HQ_ERR_NULL;
+    if (!aligned16(in) || !aligned16(out_fp8) || !aligned4(scales)) return HQ_ERR_ALIGN;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return HQ_ERR_CUDA;
+    K128Params p;
+    p.in = in;
+    p.K_out = K_out;
+    p.ngroups = M * (K_out / 128);
+    p.out = out_fp8;
+    p.scales = scales;
+    constexpr int warps_per_block = K128_THREADS / 32;
+    const int64_t pairs = (p.ngroups + 1) / 2;
+    const int64_t per_block = (int64_t)warps_per_block * K128_UNROLL;
+    const int64_t blocks_needed = (pairs + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)dev->sms * 8;
+    const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
+    launch_k128(mode, p, grid, (cudaStream_t)stream);
+    return launch_status();
+}
+
+hq_status hq_convert(int fmt, const float* in, uint8_t* out, int64_t n, void* stream) {
+    if (fmt != HQ_FMT_E4M3 && fmt != HQ_FMT_E2M1) return HQ_ERR_UNSUPPORTED;
+    if (n < 0) return HQ_ERR_SHAPE;
+    if (n == 0) return HQ_OK;
+    if (!in || !out) return HQ_ERR_NULL;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return HQ_ERR_CUDA;
+    const int64_t blocks = (n + 255) / 256;
+    const int64_t cap = (int64_t)dev->sms * 16;
+    launch_convert(fmt, in, out, n, (int)(blocks < cap ? blocks : cap), (cudaStream_t)stream);
+    return launch_status();
+}
+
+}  // extern "C"

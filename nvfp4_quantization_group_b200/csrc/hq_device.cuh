@@ -1,0 +1,224 @@
+// hq_device.cuh -- device helpers shared by the hq kernels (sm_100a).
+//
+// All floating-point steps that decide a code or a scale are written as
+// explicit round-to-nearest intrinsics (__fadd_rn, __fmul_rn, __fdiv_rn,
+// __fmaf_rn) or packed f32x2 PTX with .rn, so the compiler cannot contract
+// or reorder them; the library is also built with -fmad=false.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hq {
+
+// ------------------------------------------------------------ conversions
+// BF16 is the upper half of a binary32 word.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two FP32 values -> two E4M3 codes (saturating, nearest even): `lo` in
+// bits 0..7, `hi` in bits 8..15.  The PTX instruction places its first
+// source operand in the upper byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight FP32 values -> eight E2M1 codes packed into 32 bits, element k in
+// nibble k (element 2k low, 2k+1 high within byte k).
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3,
+                                           float v4, float v5, float v6, float v7) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return r;
+}
+
+// Single-value forms (used by the element-wise codec).
+__device__ __forceinline__ uint8_t e4m3_one(float v) { return (uint8_t)(e4m3x2(v, 0.0f) & 0xFF); }
+__device__ __forceinline__ uint8_t e2m1_one(float v) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\tcvt.u16.u8 %0, q;\n\t}"
+        : "=h"(r) : "f"(0.0f), "f"(v));
+    return (uint8_t)(r & 0xF);
+}
+
+// Value of a non-negative E4M3 code (0x00..0x7E).  Shifting the 7 code bits
+// to binary32 bit 20 gives exponent field e and mantissa m << 20, i.e.
+// (1 + m/8) * 2^(e-127) (or m * 2^-129 for e == 0); multiplying by 2^120
+// re-biases the exponent (exact: the result is a normal binary32 value).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    return __fmul_rn(__uint_as_float(code << 20), __uint_as_float(0x7B800000u));
+}
+
+// ------------------------------------------------------- packed f32x2 math
+// Two binary32 values in one 64-bit register; PTX f32x2 ops (sm_100a)
+// round each half to nearest exactly as the scalar ops would.
+typedef unsigned long long f2;
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// Two BF16 values (one 32-bit word, element 0 low) -> packed f32x2.
+__device__ __forceinline__ f2 bf16x2_to_f2(uint32_t w) { return pack2(bf16_lo(w), bf16_hi(w)); }
+
+// max(m, |a|, |b|) with NaN-skipping semantics (max.f32 returns the non-NaN
+// operand).
+__device__ __forceinline__ float absmax3(float m, float a, float b) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+    return r;
+}
+
+// ------------------------------------------------------------ Hadamard
+// Unnormalised Sylvester butterfly, stages h = 1, 2, 4, ... ascending:
+// (a, b) -> (a + b, a - b) for every pair (i, i + h) with (i & h) == 0.
+
+// In place on N scalars held in registers (N a power of two).
+template <int N>
+__device__ __forceinline__ void fwht_regs(float (&v)[N]) {
+#pragma unroll
+    for (int h = 1; h < N; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+}
+
+// The same butterfly over index i of 16 packed pairs: pair i holds element i
+// of two independent vectors, so both transforms run in one f32x2 op each.
+__device__ __forceinline__ void fwht16_x2(f2 (&v)[16]) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & h) == 0) {
+                f2 a = v[i], b = v[i + h];
+                v[i] = add2(a, b);
+                v[i + h] = sub2(a, b);
+            }
+        }
+    }
+}
+
+// -------------------------------------------------------------- FP8 rule
+// Scale of one group: max(amax, 1e-10f) * float32(1/448).
+__device__ __forceinline__ float fp8_group_scale(float amax) {
+    const float floor_ = __uint_as_float(0x2EDBE6FFu);  // 1e-10f
+    const float inv448 = __uint_as_float(0x3B124925u);  // RN(1/448)
+    return __fmul_rn(fmaxf(amax, floor_), inv448);
+}
+
+// ----------------------------------------------- correctly rounded y / b
+// The quantizers divide many numerators by one divisor b.  Instead of an
+// IEEE division per element they take r = RN(1/b) once and refine
+// q0 = RN(y * r) with two FMA remainder corrections (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990): q0 is within 1.5 ulp of y/b; one correction makes it a
+// faithful rounding, after which the remainder b*q - y is exact and the second
+// correction yields RN(y / b).  The callers pass ny = -y and nr = -r so that
+// the sign of a zero quotient comes out as IEEE division gives it.  Valid for
+// 0 < b < inf with no underflow in the remainders, which holds whenever the
+// quotient can reach a nonzero FP8/FP4 code; callers route b = inf (and
+// subnormal numerators of the NVFP4 block scale) to __fdiv_rn.
+struct Recip {
+    float b, nr;
+};
+__device__ __forceinline__ Recip make_recip(float b) { return Recip{b, -__frcp_rn(b)}; }
+
+__device__ __forceinline__ float div_rn_neg(float ny, Recip d) {
+    float q = __fmul_rn(ny, d.nr);
+    float e = __fmaf_rn(d.b, q, ny);
+    q = __fmaf_rn(e, d.nr, q);
+    e = __fmaf_rn(d.b, q, ny);
+    return __fmaf_rn(e, d.nr, q);
+}
+
+// Same, on two numerators sharing one divisor (packed f32x2).
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f2 div2_rn_neg(f2 ny, f2 b2, f2 nr2) {
+    f2 q = mul2(ny, nr2);
+    f2 e = fma2(b2, q, ny);
+    q = fma2(e, nr2, q);
+    e = fma2(b2, q, ny);
+    return fma2(e, nr2, q);
+}
+
+// RN(a / 6) for finite a >= 0.
+__device__ __forceinline__ float div6_rn(float a) {
+    if (a < 7.8886091e-31f)  // 2^-100: keep the remainders out of the subnormal range
+        return __fdiv_rn(a, 6.0f);
+    const Recip six{6.0f, -__uint_as_float(0x3E2AAAABu)};  // -RN(1/6)
+    return div_rn_neg(-a, six);
+}
+
+// --------------------------------------------------------- memory access
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t policy) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(policy));
+    return v;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+}  // namespace hq

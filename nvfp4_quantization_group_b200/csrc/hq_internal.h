@@ -1,0 +1,114 @@
+// hq_internal.h -- kernel parameter blocks and declarations shared by the
+// hq host layer (hq_api.cu) and the kernels (hq_fp8.cu, hq_nvfp4.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hq.h"
+#include "hq_device.cuh"
+
+namespace hq {
+
+// --------------------------------------------------------------- FP8 paths
+struct CatRotateParams {
+    const uint16_t* a;
+    const uint16_t* b;
+    int64_t a_row_stride, b_row_stride;
+    int a_width, b_width;
+    int64_t nvec;  // M * G vectors of 128
+    int G;
+    int rotate;    // 1: H128 / sqrt(128); 0: none
+    uint8_t* out;
+    float* scales;
+    int scale_layout;
+    int64_t scale_ld;
+};
+
+struct K128Params {
+    const void* in;
+    int64_t K_out;
+    int64_t ngroups;  // M * K_out / 128
+    uint8_t* out;
+    float* scales;
+};
+
+constexpr int K128_THREADS = 256;   // 8 warps, two K128 groups per warp step
+constexpr int K128_UNROLL = 4;      // warp steps with loads in flight
+
+int cat_rotate_blocks_per_sm();
+void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st);
+void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st);
+void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st);
+
+// exp(x) in binary32 by one fixed sequence of IEEE operations: Cody & Waite
+// reduction k = rint(x * log2(e)), r = (x - k*LN2_HI) - k*LN2_LO (two FMAs),
+// e^r by its degree-7 Taylor polynomial (Horner, FMA), times 2^k in at most
+// two exact power-of-two steps.  x > 88.8 -> +inf, x < -104 -> +0.
+__device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
+__device__ __forceinline__ float hq_exp(float x) {
+    if (isnan(x)) return x;
+    if (x > 88.8f) return __uint_as_float(0x7F800000u);
+    if (x < -104.0f) return 0.0f;
+    const float LOG2E = __uint_as_float(0x3FB8AA3Bu);
+    const float LN2_HI = __uint_as_float(0x3F317200u);
+    const float LN2_LO = __uint_as_float(0x35BFBE8Eu);
+    const float k = rintf(__fmul_rn(x, LOG2E));
+    float r = __fmaf_rn(-k, LN2_HI, x);
+    r = __fmaf_rn(-k, LN2_LO, r);
+    float p = __uint_as_float(0x39500D01u);            // RN(1/5040)
+    p = __fmaf_rn(p, r, __uint_as_float(0x3AB60B61u)); // RN(1/720)
+    p = __fmaf_rn(p, r, __uint_as_float(0x3C088889u)); // RN(1/120)
+    p = __fmaf_rn(p, r, __uint_as_float(0x3D2AAAABu)); // RN(1/24)
+    p = __fmaf_rn(p, r, __uint_as_float(0x3E2AAAABu)); // RN(1/6)
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ki = (int)k;
+    if (ki > 127) return __fmul_rn(__fmul_rn(p, pow2i(127)), pow2i(ki - 127));
+    if (ki < -126) return __fmul_rn(__fmul_rn(p, pow2i(ki + 100)), pow2i(-100));
+    return __fmul_rn(p, pow2i(ki));
+}
+
+// -(SiLU(g) * u) in binary32: SiLU(g) = g / (1 + exp(-g)) (IEEE division);
+// the product is negated through its operand (u -> -u), which rounding to
+// nearest maps to the exact negation of SiLU(g) * u.
+__device__ __forceinline__ float neg_swiglu(float g, float u) {
+    const float e = hq_exp(-g);
+    const float silu = __fdiv_rn(g, __fadd_rn(1.0f, e));
+    return __fmul_rn(silu, -u);
+}
+
+// ------------------------------------------------------------ NVFP4 path
+constexpr int NV_TILE = 128;                 // tile = 128 rows x 128 columns
+constexpr int NV_THREADS = 128;              // 4 warps, one 16x8 patch per thread
+constexpr int NV_MAX_SEG = 2 * HQ_MAX_SECTIONS;
+constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, spare
+
+// Workspace words (uint32): [0] tile counter, [1] CTAs finished, [2] error
+// word, [3] spare, then amax_row bits [S], amax_col bits [S], amax-pass tiles
+// finished per section [S].
+struct NvParams {
+    const uint16_t* x;
+    int64_t K;
+    uint8_t *row_codes, *row_sf, *col_codes, *col_sf;
+    float *amax_row, *amax_col, *sdec_row, *sdec_col;
+    uint32_t* ws;
+    int S;
+    uint32_t sign_mask;
+    uint32_t flags;
+    int col_tiles;      // K / 128
+    int nseg;           // schedule segments
+    uint32_t total_items;
+    int finalize;       // last launch of the call: publish amax/sdec, reset ws
+    int reset_counter;  // reset the tile counter / exit count at the end
+    int sec_row0[HQ_MAX_SECTIONS + 1];
+    uint32_t seg_start[NV_MAX_SEG + 1];
+    uint16_t seg_info[NV_MAX_SEG];  // section | (phase << 15); phase 0 amax, 1 cast
+};
+
+int nvfp4_blocks_per_sm();
+void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st);
+
+}  // namespace hq

@@ -1,0 +1,124 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every function include/hq.h declares, and
+reject bad arguments with the documented status before touching the GPU.
+Pointers here are fake non-null addresses: every call below fails argument
+checks, so nothing is dereferenced or launched.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_quantization_group_b200 as hq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hq.h")
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+P = ctypes.c_void_p
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    return hq.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(hq.EXPORTED)
+
+
+def test_version_and_status_strings(L):
+    assert hq.hq_version() >= 1
+    for s in range(8):
+        assert hq.status_string(s)
+    assert hq.status_string(hq.HQ_ERR_ALIGN).startswith("misaligned")
+
+
+def test_workspace_size_query():
+    assert hq.hq_group_rht_quant_workspace_size(0) == 0
+    assert hq.hq_group_rht_quant_workspace_size(hq.HQ_MAX_SECTIONS + 1) == 0
+    s1 = hq.hq_group_rht_quant_workspace_size(1)
+    s32 = hq.hq_group_rht_quant_workspace_size(32)
+    s256 = hq.hq_group_rht_quant_workspace_size(256)
+    assert s1 >= 4 and s1 % 256 == 0 and s1 <= s32 <= s256
+    assert s32 >= 4 * (4 + 3 * 32)          # counter word first, then per-section words
+
+
+def _grp(L, x=FAKE, M=256, K=256, splits=(128, 128), flags=3, ptrs=FAKE, ws=FAKE, ws_bytes=4096,
+         row_codes=None):
+    arr = (ctypes.c_int64 * len(splits))(*splits)
+    rc = FAKE if row_codes is None else row_codes
+    return L.hq_group_rht_quant(P(x), M, K, ctypes.cast(arr, P), len(splits), 0x1234, flags,
+                                P(rc), P(ptrs), P(ptrs), P(ptrs), P(ptrs), P(ptrs), P(ptrs), P(ptrs),
+                                P(ws), ws_bytes, None)
+
+
+def test_group_rht_quant_argument_errors(L):
+    assert _grp(L, flags=0) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp(L, flags=16) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp(L, x=0) == hq.HQ_ERR_NULL
+    assert _grp(L, ws=0) == hq.HQ_ERR_NULL
+    assert _grp(L, ptrs=0) == hq.HQ_ERR_NULL
+    assert _grp(L, K=200) == hq.HQ_ERR_ALIGN                       # K % 128
+    assert _grp(L, splits=(64, 192)) == hq.HQ_ERR_ALIGN            # split % 128 (fusion rule)
+    assert _grp(L, splits=(128, 256)) == hq.HQ_ERR_SHAPE           # sum != M
+    assert _grp(L, splits=(128, -128, 256)) == hq.HQ_ERR_SHAPE
+    assert _grp(L, splits=(128,) * 2 + (0,) * 300, M=256) == hq.HQ_ERR_SHAPE  # S > 256
+    assert _grp(L, ws_bytes=16) == hq.HQ_ERR_WORKSPACE
+    assert _grp(L, x=FAKE + 8) == hq.HQ_ERR_ALIGN
+    assert _grp(L, row_codes=FAKE + 4) == hq.HQ_ERR_ALIGN
+
+
+def test_cat_rotate_fp8_argument_errors(L):
+    def call(a=FAKE, a_rs=64 * 64, aw=64, b=FAKE, b_rs=64 * 64, bw=64, M=16, G=64, hn=128, out=FAKE,
+             sc=FAKE, layout=0, ld=16):
+        return L.hq_cat_rotate_fp8(P(a), a_rs, aw, P(b), b_rs, bw, M, G, hn, P(out), P(sc), layout, ld,
+                                   None, 0, None)
+    assert call(hn=64) == hq.HQ_ERR_UNSUPPORTED
+    assert call(layout=2) == hq.HQ_ERR_UNSUPPORTED
+    assert call(aw=64, bw=32) == hq.HQ_ERR_SHAPE                  # widths must sum to 128
+    assert call(M=0) == hq.HQ_OK                                   # empty: nothing to do
+    assert call(a=0) == hq.HQ_ERR_NULL
+    assert call(b=0) == hq.HQ_ERR_NULL
+    assert call(aw=60, bw=68) == hq.HQ_ERR_ALIGN
+    assert call(a_rs=64 * 64 + 4) == hq.HQ_ERR_ALIGN
+    assert call(a_rs=64) == hq.HQ_ERR_SHAPE                        # stride shorter than G groups
+    assert call(layout=1, ld=8) == hq.HQ_ERR_SHAPE                 # transposed ld < M
+    assert call(out=FAKE + 1) == hq.HQ_ERR_ALIGN
+
+
+def test_swiglu_fp8_k128_argument_errors(L):
+    def call(mode=0, inp=FAKE, M=4, K=256, out=FAKE, sc=FAKE):
+        return L.hq_swiglu_fp8_k128(mode, P(inp), M, K, P(out), P(sc), None, 0, None)
+    assert call(mode=3) == hq.HQ_ERR_UNSUPPORTED
+    assert call(K=200) == hq.HQ_ERR_ALIGN
+    assert call(M=-1) == hq.HQ_ERR_SHAPE
+    assert call(M=0) == hq.HQ_OK
+    assert call(inp=0) == hq.HQ_ERR_NULL
+    assert call(inp=FAKE + 8) == hq.HQ_ERR_ALIGN
+    assert call(sc=FAKE + 2) == hq.HQ_ERR_ALIGN
+
+
+def test_convert_and_workspace_argument_errors(L):
+    assert L.hq_convert(2, P(FAKE), P(FAKE), 10, None) == hq.HQ_ERR_UNSUPPORTED
+    assert L.hq_convert(0, P(FAKE), P(FAKE), -1, None) == hq.HQ_ERR_SHAPE
+    assert L.hq_convert(0, P(FAKE), P(FAKE), 0, None) == hq.HQ_OK
+    assert L.hq_convert(0, None, P(FAKE), 10, None) == hq.HQ_ERR_NULL
+    assert L.hq_workspace_init(None, 256, None) == hq.HQ_ERR_NULL
+    assert L.hq_workspace_init(P(FAKE + 4), 256, None) == hq.HQ_ERR_ALIGN
+    err = ctypes.c_uint32(0)
+    assert L.hq_get_error(None, 256, ctypes.byref(err), None) == hq.HQ_ERR_NULL
+    assert L.hq_get_error(P(FAKE), 8, ctypes.byref(err), None) == hq.HQ_ERR_WORKSPACE

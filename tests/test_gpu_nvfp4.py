@@ -1,0 +1,176 @@
+"""GPU parity: grouped RHT16 + NVFP4 cast (hq_group_rht_quant) against the
+oracle -- small ragged section mixes, both schedules, direction flags,
+workspace rest state, repeated calls, guard bands, and the full dense and
+grouped-MoE workloads."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from _compare import assert_bits_equal, assert_fp4_codes
+
+pytestmark = pytest.mark.gpu
+
+ROW_KEYS = ("row_codes", "row_sf", "amax_row", "sdec_row")
+COL_KEYS = ("col_codes", "col_sf", "amax_col", "sdec_col")
+GUARD = 4096
+
+
+def _bf16_dev(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).cuda()
+
+
+def _guarded_outputs(hq, M, K, S, flags):
+    """Outputs carved from buffers poisoned with 0xA5 and followed by a guard band."""
+    bufs, out = {}, {}
+    shapes = {}
+    if flags & hq.HQ_ROWWISE:
+        shapes.update(row_codes=(M * K // 2, torch.uint8), row_sf=(M * K // 16, torch.uint8),
+                      amax_row=(S, torch.float32), sdec_row=(S, torch.float32))
+    if flags & hq.HQ_COLWISE:
+        shapes.update(col_codes=(M * K // 2, torch.uint8), col_sf=(M * K // 16, torch.uint8),
+                      amax_col=(S, torch.float32), sdec_col=(S, torch.float32))
+    for k, (n, dt) in shapes.items():
+        nbytes = n * (4 if dt == torch.float32 else 1)
+        raw = torch.full((nbytes + GUARD,), 0xA5, dtype=torch.uint8, device="cuda")
+        bufs[k] = raw
+        out[k] = raw[:nbytes].view(dt)
+    if "row_codes" in out:
+        out["row_codes"] = out["row_codes"].view(M, K // 2)
+        out["row_sf"] = out["row_sf"].view(M, K // 16)
+    return out, bufs
+
+
+def _run(hq, x, splits, mask, flags, ws=None):
+    M, K = x.shape
+    S = len(splits)
+    if ws is None:
+        ws = hq.new_workspace(S)
+    out, bufs = _guarded_outputs(hq, M, K, S, flags)
+    hq.group_rht_quant(_bf16_dev(x), splits, mask, flags, ws=ws, out=out)
+    torch.cuda.synchronize()
+    for k, raw in bufs.items():
+        assert torch.all(raw[-GUARD:] == 0xA5), f"guard band of {k} overwritten"
+    return {k: v.cpu().numpy() for k, v in out.items()}, ws
+
+
+def _check(got, want, x, splits, mask, flags):
+    pre = {}
+
+    def pre_of(key):
+        if key not in pre:
+            pre.update(oracle.group_rht_quant(x, splits, mask, flags, want_pre=True))
+        return pre[key]
+
+    if flags & oracle.ROWWISE:
+        assert_bits_equal(got["amax_row"], want["amax_row"], "amax_row")
+        assert_bits_equal(got["sdec_row"], want["sdec_row"], "sdec_row")
+        assert_bits_equal(got["row_sf"], want["row_sf"], "row_sf")
+        assert_fp4_codes(got["row_codes"], want["row_codes"], lambda: pre_of("row_pre"), "row codes")
+    if flags & oracle.COLWISE:
+        assert_bits_equal(got["amax_col"], want["amax_col"], "amax_col")
+        assert_bits_equal(got["sdec_col"], want["sdec_col"], "sdec_col")
+        assert_bits_equal(got["col_sf"], want["col_sf"], "col_sf")
+        assert_fp4_codes(got["col_codes"], want["col_codes"], lambda: pre_of("col_pre"), "col codes")
+
+
+def _case(seed, K, splits, scale_sections=True, outliers=0.002):
+    M = sum(splits)
+    x = S.normal_bf16(seed, (M, K))
+    if scale_sections:
+        xf = S.bf16_bits_to_f32(x).copy()
+        r0 = 0
+        for i, m in enumerate(splits):
+            xf[r0:r0 + m] *= np.float32(2.0 ** ((i % 7) - 3))
+            r0 += m
+        x = S.f32_to_bf16_bits(xf)
+    if outliers:
+        x = S.with_outliers_bf16(x, seed + 1, p=outliers)
+    return x
+
+
+@pytest.mark.parametrize("flags_extra", [0, 8])
+def test_small_sections_both_directions(hq, flags_extra):
+    splits = [128, 0, 256, 128, 0, 384]
+    x = _case(401, 256, splits)
+    mask = 0xA5C3
+    flags = hq.HQ_ROWWISE | hq.HQ_COLWISE
+    got, _ = _run(hq, x, splits, mask, flags | flags_extra)
+    _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
+
+
+@pytest.mark.parametrize("flags", [1, 2])
+def test_single_direction(hq, flags):
+    splits = [256, 128]
+    x = _case(411, 384, splits)
+    got, _ = _run(hq, x, splits, 0x0F0F, flags)
+    _check(got, oracle.group_rht_quant(x, splits, 0x0F0F, flags), x, splits, 0x0F0F, flags)
+    assert set(got) == set(ROW_KEYS if flags == 1 else COL_KEYS)
+
+
+def test_many_sections_random_splits_and_masks(hq):
+    splits = S.random_splits(421, total_units=24, sections=40)
+    x = _case(422, 512, splits)
+    for mask in (0x0000, 0xFFFF, S.sign_mask16(423)):
+        got, _ = _run(hq, x, splits, mask, 3)
+        _check(got, oracle.group_rht_quant(x, splits, mask, 3), x, splits, mask, 3)
+
+
+def test_all_sections_empty_and_zero_data(hq):
+    splits = [0, 0, 0]
+    x = np.zeros((0, 128), dtype=np.uint16)
+    got, _ = _run(hq, x, splits, 0x1234, 3)
+    assert np.all(got["amax_row"] == 0) and np.all(got["sdec_row"] == 1)
+    assert np.all(got["amax_col"] == 0) and np.all(got["sdec_col"] == 1)
+    splits = [128, 128]
+    x = np.zeros((256, 128), dtype=np.uint16)
+    x[128:] = S.normal_bf16(431, (128, 128))
+    got, _ = _run(hq, x, splits, 0x00FF, 3)
+    _check(got, oracle.group_rht_quant(x, splits, 0x00FF, 3), x, splits, 0x00FF, 3)
+
+
+def test_workspace_returns_to_rest_and_calls_repeat(hq):
+    splits = [128, 256, 0, 128]
+    x = _case(441, 256, splits)
+    ws = hq.new_workspace(len(splits))
+    first, ws = _run(hq, x, splits, 0x5A5A, 3, ws=ws)
+    assert torch.count_nonzero(ws).item() == 0, "workspace not back in its rest state"
+    for extra in (0, 8, 0):
+        again, ws = _run(hq, x, splits, 0x5A5A, 3 | extra, ws=ws)
+        for k in first:
+            assert_bits_equal(again[k], first[k], k)
+        assert torch.count_nonzero(ws).item() == 0
+    assert hq.hq_get_error(ws) == 0
+
+
+def test_extreme_magnitudes(hq):
+    splits = [128, 128, 128]
+    xf = S.bf16_bits_to_f32(S.normal_bf16(451, (384, 256))).copy()
+    xf[:128] *= np.float32(1e-30)      # tiny section
+    xf[128:256] *= np.float32(1e30)    # huge section
+    xf[256:, :16] = 0.0                # zero blocks inside a normal section
+    x = S.f32_to_bf16_bits(xf)
+    got, _ = _run(hq, x, splits, 0x8001, 3)
+    _check(got, oracle.group_rht_quant(x, splits, 0x8001, 3), x, splits, 0x8001, 3)
+
+
+@pytest.mark.slow
+def test_dense_nvfp4_8192x4096(hq):
+    seed = S.SEEDS["dense_nvfp4"]
+    x = S.with_outliers_bf16(S.normal_bf16(seed, (8192, 4096)), seed + 1, p=0.001, factor=50.0)
+    mask = S.sign_mask16(seed)
+    got, _ = _run(hq, x, [8192], mask, 3)
+    _check(got, oracle.group_rht_quant(x, [8192], mask, 3), x, [8192], mask, 3)
+
+
+@pytest.mark.slow
+def test_grouped_moe_16384x7168(hq):
+    seed = S.SEEDS["grouped_moe"]
+    x = S.normal_bf16(seed, (16384, 7168))
+    splits = S.moe_splits(seed)
+    mask = S.sign_mask16(seed)
+    got, _ = _run(hq, x, splits, mask, 3)
+    _check(got, oracle.group_rht_quant(x, splits, mask, 3), x, splits, mask, 3)
