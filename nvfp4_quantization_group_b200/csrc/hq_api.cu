@@ -101,8 +101,9 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
     if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
     if (!split_rows || !ws) return HQ_ERR_NULL;
-    if (do_row && (!row_codes || !row_sf || !amax_row || !sdec_row)) return HQ_ERR_NULL;
-    if (do_col && (!col_codes || !col_sf || !amax_col || !sdec_col)) return HQ_ERR_NULL;
+    // code and block-scale buffers are empty (and may be NULL) when M == 0
+    if (do_row && (!amax_row || !sdec_row || (M > 0 && (!row_codes || !row_sf)))) return HQ_ERR_NULL;
+    if (do_col && (!amax_col || !sdec_col || (M > 0 && (!col_codes || !col_sf)))) return HQ_ERR_NULL;
     if (S < 1 || S > HQ_MAX_SECTIONS || M < 0 || K <= 0) return HQ_ERR_SHAPE;
     if (M > 0 && !x) return HQ_ERR_NULL;
     if (K % NV_TILE != 0) return HQ_ERR_ALIGN;
@@ -118,7 +119,7 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     if (do_row && (!aligned16(row_codes) || !aligned16(row_sf) || !aligned4(amax_row) || !aligned4(sdec_row)))
         return HQ_ERR_ALIGN;
     if (do_col && (!aligned16(col_codes) || !aligned16(col_sf) || !aligned4(amax_col) || !aligned4(sdec_col)))
-        return HQ_ERR_ALIGN;
+        return HQ_ERR_ALIGN;  // (NULL is 16-byte aligned: empty buffers pass)
     if (ws_bytes < hq_group_rht_quant_workspace_size(S)) return HQ_ERR_WORKSPACE;
     const DeviceInfo* dev = device_info();
     if (!dev) return HQ_ERR_CUDA;

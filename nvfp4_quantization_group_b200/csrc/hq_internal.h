@@ -84,11 +84,12 @@ __device__ __forceinline__ float neg_swiglu(float g, float u) {
 constexpr int NV_TILE = 128;                 // tile = 128 rows x 128 columns
 constexpr int NV_THREADS = 128;              // 4 warps, one 16x8 patch per thread
 constexpr int NV_MAX_SEG = 2 * HQ_MAX_SECTIONS;
-constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, spare
+constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abort
 
-// Workspace words (uint32): [0] tile counter, [1] CTAs finished, [2] error
-// word, [3] spare, then amax_row bits [S], amax_col bits [S], amax-pass tiles
-// finished per section [S].
+// Workspace words (uint32): [0] tile counter, [1] CTAs finished, [2] sticky
+// error word (cleared by hq_get_error), [3] abort flag of the running call,
+// then amax_row bits [S], amax_col bits [S], amax-pass tiles finished per
+// section [S].  All but [2] are zero between calls.
 struct NvParams {
     const uint16_t* x;
     int64_t K;

@@ -20,7 +20,7 @@ namespace hq {
 
 namespace {
 
-constexpr uint32_t SPIN_LIMIT = 1u << 21;  // x >= 64 ns: bounded wait (~0.1-1 s)
+constexpr uint32_t SPIN_LIMIT = 1u << 20;  // polls of >= 64 ns + a load: bounded wait of ~0.1-1 s
 
 struct NvShared {
     float enc_row[128];  // S_enc_row / value(sf) for every E4M3 code sf
@@ -55,7 +55,8 @@ __global__ void __launch_bounds__(NV_THREADS) nvfp4_group_kernel(const __grid_co
     __shared__ NvShared sh;
     uint32_t* const counter = p.ws;
     uint32_t* const exit_count = p.ws + 1;
-    uint32_t* const err = p.ws + 2;
+    uint32_t* const err = p.ws + 2;        // sticky, read by hq_get_error
+    uint32_t* const abort_flag = p.ws + 3; // this call only; cleared at exit
     uint32_t* const amax_row_ws = p.ws + NV_WS_HEADER;
     uint32_t* const amax_col_ws = amax_row_ws + p.S;
     uint32_t* const done_ws = amax_col_ws + p.S;
@@ -109,8 +110,13 @@ __global__ void __launch_bounds__(NV_THREADS) nvfp4_group_kernel(const __grid_co
                 const uint32_t target = (uint32_t)trows * (uint32_t)p.col_tiles;
                 uint32_t spins = 0;
                 while (ld_acquire(done_ws + s) < target) {
-                    if (++spins > SPIN_LIMIT || *(volatile uint32_t*)err != 0) {
+                    if (*(volatile uint32_t*)abort_flag != 0) {  // another CTA gave up already
+                        sh.abort = 1;
+                        break;
+                    }
+                    if (++spins > SPIN_LIMIT) {
                         atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
+                        atomicExch(abort_flag, 1u);
                         sh.abort = 1;
                         break;
                     }
@@ -284,6 +290,7 @@ __global__ void __launch_bounds__(NV_THREADS) nvfp4_group_kernel(const __grid_co
     if (tid == 0 && p.reset_counter) {
         *counter = 0;
         *exit_count = 0;
+        *abort_flag = 0;
     }
 }
 

@@ -174,3 +174,30 @@ def test_grouped_moe_16384x7168(hq):
     mask = S.sign_mask16(seed)
     got, _ = _run(hq, x, splits, mask, 3)
     _check(got, oracle.group_rht_quant(x, splits, mask, 3), x, splits, mask, 3)
+
+
+def test_bounded_wait_reports_timeout_and_recovers(hq):
+    """A workspace outside its rest state makes the cast tile's wait run out:
+    with the tile counter starting at 1, item 0 (the section's only amax tile)
+    is never claimed, so its cast tile (item 1) waits for an amax that never
+    comes.  The call ends by itself after the bounded spin, hq_get_error
+    reports HQ_ERR_TIMEOUT, the workspace is back at rest and the next call is
+    correct."""
+    splits = [128]
+    x = _case(461, 128, splits)
+    ws = hq.new_workspace(1)
+    words = ws.view(torch.int32)
+    words[0] = 1                     # tile counter
+    out = hq.group_outputs(128, 128, 1)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    hq.group_rht_quant(_bf16_dev(x), splits, 0x1111, 3, ws=ws, out=out)
+    t1.record()
+    torch.cuda.synchronize()
+    assert t0.elapsed_time(t1) < 30000
+    assert hq.hq_get_error(ws) == hq.HQ_ERR_TIMEOUT
+    assert torch.count_nonzero(ws).item() == 0
+    got, _ = _run(hq, x, splits, 0x1111, 3, ws=ws)
+    _check(got, oracle.group_rht_quant(x, splits, 0x1111, 3), x, splits, 0x1111, 3)
+    assert hq.hq_get_error(ws) == 0
