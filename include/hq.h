@@ -138,7 +138,8 @@ hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *strea
  *  col_sf     uint8 [M*K/16]     per section s: [K, M_s/16] at byte K*r0/16
  *  amax_row, sdec_row  float [S] (HQ_ROWWISE)
  *  amax_col, sdec_col  float [S] (HQ_COLWISE)
- *  Pointers of a direction not requested may be NULL.
+ *  Pointers of a direction not requested may be NULL, and so may the code
+ *  and block-scale buffers when M == 0.
  *
  *  ws, ws_bytes  caller workspace, >= hq_group_rht_quant_workspace_size(S),
  *                16-byte aligned, in the rest state (hq_workspace_init).
