@@ -157,6 +157,32 @@ hq_status hq_group_rht_quant(const void *x, int64_t M, int64_t K,
                              void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * hq_group_rht_quant without a caller workspace, for callers that cannot
+ * allocate device memory where they quantize (code running while a CUDA
+ * graph is captured, plugins whose host framework owns all device memory,
+ * allocation-free runtimes).  The paper has no counterpart.
+ *
+ * Arguments, outputs and errors are those of hq_group_rht_quant without
+ * ws / ws_bytes.  The scratch words live in a fixed array inside the library
+ * (3328 bytes, room for HQ_MAX_SECTIONS = 256 sections; S > 256 returns
+ * HQ_ERR_SHAPE), present on every GPU that loads the library until the
+ * process exits.  The call allocates nothing: it clears the array with an
+ * enqueued memset and launches the kernel.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress) and so should come
+ * before any stream capture.  All calls on a device share the one array:
+ * calls that overlap on the GPU (different streams without ordering) race
+ * and give wrong results.  A bounded device wait that gives up is not
+ * reported by this entry point (there is no workspace to read it from).
+ */
+hq_status hq_group_rht_quant_noalloc(const void *x, int64_t M, int64_t K,
+                                     const int64_t *split_rows, int S, uint16_t sign_mask,
+                                     unsigned flags,
+                                     uint8_t *row_codes, uint8_t *row_sf,
+                                     uint8_t *col_codes, uint8_t *col_sf,
+                                     float *amax_row, float *amax_col,
+                                     float *sdec_row, float *sdec_col, void *stream);
+
+/*
  * Concatenate -> 128-point Hadamard rotation -> FP8 E4M3 1x128 quantization
  * [DSA] (the DSA indexer's q/k preparation), with the scale rule of [QMOE].
  *

@@ -30,7 +30,8 @@ HQ_MAX_SECTIONS = 256
 
 EXPORTED = (
     "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
-    "hq_get_error", "hq_group_rht_quant", "hq_cat_rotate_fp8", "hq_swiglu_fp8_k128", "hq_convert",
+    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8", "hq_swiglu_fp8_k128",
+    "hq_convert",
 )
 
 
@@ -65,6 +66,9 @@ def lib() -> ctypes.CDLL:
         L.hq_group_rht_quant.restype = c_int
         L.hq_group_rht_quant.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
                                          P, P, P, P, P, P, P, P, P, sz, P]
+        L.hq_group_rht_quant_noalloc.restype = c_int
+        L.hq_group_rht_quant_noalloc.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
+                                                 P, P, P, P, P, P, P, P, P]
         L.hq_cat_rotate_fp8.restype = c_int
         L.hq_cat_rotate_fp8.argtypes = [P, i64, c_int, P, i64, c_int, i64, c_int, c_int,
                                         P, P, c_int, i64, P, sz, P]
@@ -129,6 +133,17 @@ def hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, row_codes, row_
                                     int(sign_mask) & 0xFFFF, int(flags), _p(row_codes), _p(row_sf),
                                     _p(col_codes), _p(col_sf), _p(amax_row), _p(amax_col), _p(sdec_row),
                                     _p(sdec_col), _p(ws), ws_bytes, _stream(stream)), "hq_group_rht_quant")
+
+
+def hq_group_rht_quant_noalloc(x, M, K, split_rows, S, sign_mask, flags, row_codes, row_sf, col_codes, col_sf,
+                               amax_row, amax_col, sdec_row, sdec_col, stream=None) -> None:
+    """hq_group_rht_quant with the library's fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    splits = (ctypes.c_int64 * len(split_rows))(*[int(v) for v in split_rows])
+    _check(lib().hq_group_rht_quant_noalloc(_p(x), int(M), int(K), ctypes.cast(splits, ctypes.c_void_p), int(S),
+                                            int(sign_mask) & 0xFFFF, int(flags), _p(row_codes), _p(row_sf),
+                                            _p(col_codes), _p(col_sf), _p(amax_row), _p(amax_col), _p(sdec_row),
+                                            _p(sdec_col), _stream(stream)), "hq_group_rht_quant_noalloc")
 
 
 def hq_cat_rotate_fp8(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, out_fp8, scales,
