@@ -1,6 +1,7 @@
 // hq_api.cu -- the extern "C" entry points of include/hq.h: argument checks,
 // kernel parameter blocks, grid sizing and launches.  No allocation, no
 // synchronization (hq_get_error excepted), no environment reads.
+#include <cudaTypedefs.h>
 #include <string.h>
 
 #include <mutex>
@@ -45,6 +46,36 @@ inline hq_status launch_status() {
 }
 
 size_t nv_ws_words(int S) { return (size_t)NV_WS_HEADER + 3 * (size_t)S; }
+
+// The driver's tensor-map encoder, reached once through the runtime (no link
+// against the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// x (BF16 [M, K], rows of K elements) viewed as [M/16][16][K]: 16-row block,
+// row in block, column.  Boxes of 64 columns x 8 blocks x 16 rows land
+// row-in-block major with the 128-byte swizzle.
+bool encode_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)(M / 16), 16};
+    const cuuint64_t strides[2] = {(cuuint64_t)(16 * K * 2), (cuuint64_t)(K * 2)};  // bytes, dims 1 and 2
+    const cuuint32_t box[3] = {64, 8, 16};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -129,6 +160,7 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     memset(&p, 0, sizeof p);
     p.x = static_cast<const uint16_t*>(x);
     p.K = K;
+    if (M > 0 && K > 0 && !encode_x_map(&p.tmap, x, M, K)) return HQ_ERR_CUDA;
     p.row_codes = row_codes; p.row_sf = row_sf; p.col_codes = col_codes; p.col_sf = col_sf;
     p.amax_row = amax_row; p.amax_col = amax_col; p.sdec_row = sdec_row; p.sdec_col = sdec_col;
     p.ws = static_cast<uint32_t*>(ws);
@@ -155,22 +187,38 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     };
     cudaStream_t st = (cudaStream_t)stream;
     const int max_grid = dev->sms * (dev->nv_blocks_per_sm > 0 ? dev->nv_blocks_per_sm : 1);
+    auto grid_for = [&](uint32_t items) {
+        return (int)(items < (uint32_t)max_grid ? (items > 0 ? items : 1) : (uint32_t)max_grid);
+    };
     auto launch = [&](NvParams& q, uint32_t items) -> hq_status {
         q.seg_start[q.nseg] = items;
         q.total_items = items;
-        const int grid = (int)(items < (uint32_t)max_grid ? (items > 0 ? items : 1) : (uint32_t)max_grid);
-        launch_nvfp4(q, grid, st);
+        launch_nvfp4(q, grid_for(items), st);
         return launch_status();
     };
 
     if (!(flags & HQ_TWO_PASS)) {
-        // A(s0) A(s1) C(s0) A(s2) C(s1) ... C(s_last)
-        uint32_t next = 0;
+        // One launch.  The cast segment of a section follows its amax segment
+        // once `lag` more tiles have been scheduled (the tiles the grid holds
+        // in flight), so its amax is normally complete when its first tile is
+        // claimed and its rows are still in L2.
+        uint32_t all = 0;
+        for (int k = 0; k < nlive; ++k) all += 2 * tiles_of(live[k]);
+        const uint32_t lag = (uint32_t)grid_for(all) * (uint32_t)nvfp4_tiles_in_flight_per_cta();
+        uint32_t next = 0, a_end[HQ_MAX_SECTIONS];
+        int pend = 0;  // next section whose cast segment is still to be scheduled
         for (int k = 0; k < nlive; ++k) {
             add_seg(p, live[k], 0, next);
-            if (k >= 1) add_seg(p, live[k - 1], 1, next);
+            a_end[k] = next;
+            while (pend < k && next - a_end[pend] >= lag) {
+                add_seg(p, live[pend], 1, next);
+                ++pend;
+            }
         }
-        if (nlive > 0) add_seg(p, live[nlive - 1], 1, next);
+        while (pend < nlive) {
+            add_seg(p, live[pend], 1, next);
+            ++pend;
+        }
         p.finalize = 1;
         p.reset_counter = 1;
         return launch(p, next);

@@ -2,6 +2,7 @@
 // hq host layer (hq_api.cu) and the kernels (hq_fp8.cu, hq_nvfp4.cu).
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (types only: the encoder is reached through the runtime)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -82,7 +83,9 @@ __device__ __forceinline__ float neg_swiglu(float g, float u) {
 
 // ------------------------------------------------------------ NVFP4 path
 constexpr int NV_TILE = 128;                 // tile = 128 rows x 128 columns
-constexpr int NV_THREADS = 128;              // 4 warps, one 16x8 patch per thread
+constexpr int NV_CONSUMER_WARPS = 16;        // compute warps of a CTA
+constexpr int NV_THREADS = 32 * (NV_CONSUMER_WARPS + 1);  // + the producer warp
+constexpr int NV_STAGES = 4;                 // shared-memory tile buffers per CTA
 constexpr int NV_MAX_SEG = 2 * HQ_MAX_SECTIONS;
 constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abort
 
@@ -91,6 +94,7 @@ constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abor
 // then amax_row bits [S], amax_col bits [S], amax-pass tiles finished per
 // section [S].  All but [2] are zero between calls.
 struct NvParams {
+    CUtensorMap tmap;   // x as [M/16][16][K] BF16 blocks, 64 x 8 x 16 boxes, 128-byte swizzle
     const uint16_t* x;
     int64_t K;
     uint8_t *row_codes, *row_sf, *col_codes, *col_sf;
@@ -110,6 +114,7 @@ struct NvParams {
 };
 
 int nvfp4_blocks_per_sm();
+int nvfp4_tiles_in_flight_per_cta();  // buffers + the claims in flight
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st);
 
 }  // namespace hq
