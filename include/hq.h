@@ -86,9 +86,10 @@ const char *hq_status_string(hq_status s);
 /*
  * Workspace bytes hq_group_rht_quant needs for `num_sections` sections
  * (1 <= num_sections <= HQ_MAX_SECTIONS; 0 otherwise).  The first 4 bytes
- * are the tile-scheduler counter of [GRP]; per-section amax accumulators,
- * completion counters and an error word follow.  The size query is the
- * reviewers' proposal in [GRP].
+ * are the tile-scheduler counter of [GRP]; an error word, per-section amax
+ * accumulators, completion counters and 64-bit section ready records (the
+ * section encode scales, written once the section's amax is complete)
+ * follow.  The size query is the reviewers' proposal in [GRP].
  */
 size_t hq_group_rht_quant_workspace_size(int num_sections);
 
@@ -164,7 +165,7 @@ hq_status hq_group_rht_quant(const void *x, int64_t M, int64_t K,
  *
  * Arguments, outputs and errors are those of hq_group_rht_quant without
  * ws / ws_bytes.  The scratch words live in a fixed array inside the library
- * (3328 bytes, room for HQ_MAX_SECTIONS = 256 sections; S > 256 returns
+ * (5376 bytes, room for HQ_MAX_SECTIONS = 256 sections; S > 256 returns
  * HQ_ERR_SHAPE), present on every GPU that loads the library until the
  * process exits.  The call allocates nothing: it clears the array with an
  * enqueued memset and launches the kernel.  The first call on a device looks

@@ -45,7 +45,9 @@ inline hq_status launch_status() {
     return cudaPeekAtLastError() == cudaSuccess ? HQ_OK : (cudaGetLastError(), HQ_ERR_CUDA);
 }
 
-size_t nv_ws_words(int S) { return (size_t)NV_WS_HEADER + 3 * (size_t)S; }
+// header, amax_row[S], amax_col[S], done[S], then (8-byte aligned) the 64-bit
+// section ready records[S]
+size_t nv_ws_words(int S) { return (((size_t)NV_WS_HEADER + 3 * (size_t)S + 1) & ~(size_t)1) + 2 * (size_t)S; }
 
 // The driver's tensor-map encoder, reached once through the runtime (no link
 // against the driver library).

@@ -83,9 +83,15 @@ __device__ __forceinline__ float neg_swiglu(float g, float u) {
 
 // ------------------------------------------------------------ NVFP4 path
 constexpr int NV_TILE = 128;                 // tile = 128 rows x 128 columns
-constexpr int NV_CONSUMER_WARPS = 16;        // compute warps of a CTA
+#ifndef HQ_NV_CONSUMER_WARPS
+#define HQ_NV_CONSUMER_WARPS 8
+#define HQ_NV_STAGES 3
+#define HQ_NV_CTAS_PER_SM 2
+#endif
+constexpr int NV_CONSUMER_WARPS = HQ_NV_CONSUMER_WARPS;  // compute warps of a CTA (divides 16)
 constexpr int NV_THREADS = 32 * (NV_CONSUMER_WARPS + 1);  // + the producer warp
-constexpr int NV_STAGES = 4;                 // shared-memory tile buffers per CTA
+constexpr int NV_STAGES = HQ_NV_STAGES;                  // shared-memory tile buffers per CTA
+constexpr int NV_CTAS_PER_SM = HQ_NV_CTAS_PER_SM;        // resident CTAs the kernel is built for
 constexpr int NV_MAX_SEG = 2 * HQ_MAX_SECTIONS;
 constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abort
 

@@ -4,8 +4,9 @@
 // scale factors, tile scheduler driven by a 4-byte caller workspace; PR #2555
 // review: the RHT'd columnwise output is the transposed tensor).
 //
-// One persistent kernel, one CTA per SM: a producer warp and 16 compute
-// warps around a ring of shared-memory tile buffers (128 x 128 BF16 each).
+// One persistent kernel, two CTAs per SM (each its own TMA stream): per CTA a
+// producer warp and 8 compute warps around a ring of 3 shared-memory tile
+// buffers (128 x 128 BF16 each).
 //
 //  * The producer claims 128x128 tiles from the workspace's tile counter (two
 //    claims in flight) and writes a small header per buffer.  Before the
@@ -25,11 +26,12 @@
 // tile depends only on tiles claimed before it, and compute warps never wait
 // on the producer's section wait, so the schedule cannot deadlock.
 //
-// Work split of a tile among the 16 compute warps (w) and their lanes (l):
-//  * rowwise: warp w owns rows 8w..8w+7; lane l takes row 8w + l/8 (+4) and
+// Work split of a tile into 16 parts (w), shared out among the compute warps
+// (a warp takes parts w, w + 8), and their lanes (l):
+//  * rowwise: part w is rows 8w..8w+7; lane l takes row 8w + l/8 (+4) and
 //    16-column block l%8: two 16-byte shared loads (lanes of blocks 4..7
 //    load their odd chunk first), no cross-lane traffic.
-//  * columnwise: warp w owns columns 8w..8w+7 (4 BF16 pairs); lane l takes
+//  * columnwise: part w is columns 8w..8w+7 (4 BF16 pairs); lane l takes
 //    pair 4w + l/8 and 16-row block l%8: 16 four-byte shared loads, the
 //    16-point transform of two columns in packed FP32, and two 8-byte
 //    stores; the 8 lanes of a pair write 64 contiguous bytes of the
@@ -47,14 +49,16 @@ namespace hq {
 namespace {
 
 constexpr uint32_t SPIN_LIMIT = 1u << 20;  // section polls of >= 64 ns + a load: ~0.1-1 s
-constexpr uint32_t MBAR_LIMIT = 1u << 22;  // barrier polls: far above the section wait
+constexpr uint32_t MBAR_LIMIT = 1u << 22;  // barrier sleeps of <= 1 us: far above the section wait
 constexpr int NCW = NV_CONSUMER_WARPS;
 constexpr int NST = NV_STAGES;
 constexpr int TILE_BYTES = NV_TILE * NV_TILE * 2;
 
-constexpr uint32_t H_VALID = 1u, H_CAST = 2u, H_GAVE_UP = 4u, H_FOLD = 8u;
+// header flags; H_SLOW_R / H_SLOW_C: the section encode scale is outside
+// [2^-100, 2^100], where the per-block division takes the slow exact path
+constexpr uint32_t H_VALID = 1u, H_CAST = 2u, H_GAVE_UP = 4u, H_FOLD = 8u, H_SLOW_R = 16u, H_SLOW_C = 32u;
 
-struct StageHdr {
+struct alignas(16) StageHdr {  // 48 bytes, moved as three 16-byte words
     int64_t row0;      // first global row of the tile
     int32_t col0;      // first column
     int32_t s;         // section
@@ -62,19 +66,19 @@ struct StageHdr {
     int32_t ms;        // rows of the section
     int32_t row_in_sec0;  // tile's first row inside the section
     uint32_t flags;    // H_*
-    float senc_r, senc_c;  // section encode scales (cast tiles)
-    int32_t pad;
+    float senc_r;      // section encode scale, rowwise (cast tiles)
+    float senc_c;      // columnwise
+    float senc_cq;     // numerator of the columnwise block encode factor: senc_c, times 0.25 when H_FOLD
 };
 
 struct NvShared {
-    float enc_row[NST][128];  // S_enc_row / value(sf) for every E4M3 code sf
-    float enc_col[NST][128];  // S_enc_col / value(sf), times 0.25 when folded
+    float2 vr[128];  // per E4M3 code: {value, -RN(1 / value)}; {0, -0} for codes 0 and 127
     StageHdr hdr[NST];
     uint32_t acc_row[NST], acc_col[NST], acc_cnt[NST];  // amax tiles: CTA partial maxima
-    int32_t tab_section[NST];  // section whose tables the buffer holds (producer only)
     uint32_t seg_start[NV_MAX_SEG + 1];  // copies of the schedule (parameter space is slow
     uint16_t seg_info[NV_MAX_SEG];       //   to index dynamically)
     int32_t sec_row0[HQ_MAX_SECTIONS + 1];
+    uint32_t sec_magic[HQ_MAX_SECTIONS];  // floor((2^32 - 1) / row tiles of the section)
     uint64_t full[NST], empty[NST];
     uint32_t last;  // this CTA is the last to leave
 };
@@ -166,9 +170,16 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
     t.r0s = sh.sec_row0[t.s];
     t.ms = sh.sec_row0[t.s + 1] - t.r0s;
     t.trows = t.ms / NV_TILE;
-    t.row_in_sec0 = (int)(local % (uint32_t)t.trows) * NV_TILE;
+    // local = q * trows + r by multiply-high and at most two corrections
+    uint32_t q = __umulhi(local, sh.sec_magic[t.s]);
+    uint32_t r = local - q * (uint32_t)t.trows;
+    while (r >= (uint32_t)t.trows) {
+        ++q;
+        r -= (uint32_t)t.trows;
+    }
+    t.row_in_sec0 = (int)r * NV_TILE;
     t.row0 = (int64_t)t.r0s + t.row_in_sec0;
-    t.col0 = (int)(local / (uint32_t)t.trows) * NV_TILE;
+    t.col0 = (int)q * NV_TILE;
     return t;
 }
 
@@ -176,86 +187,132 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
 
 namespace {
 
-// Header (and, for a cast tile, the section wait and the encode tables) of
-// buffer st for `tile`; returns the header flags.
-__device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, NvShared& sh, StageHdr& h, int st, uint32_t tile,
-                                           int lane, int& seg, int& cached_s, uint32_t& c_fl, uint32_t& gave_up,
-                                           float& c_sr, float& c_sc) {
-    uint32_t* const err = p.ws + 2;
-    uint32_t* const abort_flag = p.ws + 3;
-    const uint32_t* const amax_row_ws = p.ws + NV_WS_HEADER;
-    const uint32_t* const amax_col_ws = amax_row_ws + p.S;
-    const uint32_t* const done_ws = amax_col_ws + p.S;
-    {
-        const TileInfo t = decode(p, sh, tile, seg);
-        uint32_t fl = H_VALID;
-        if (t.phase == 1) {
-            fl |= H_CAST;
-            if (t.s != cached_s) {
-                // ---- wait (bounded) until every amax tile of the section is in
-                uint32_t f = 0u;
-                float sr = 1.0f, sc = 1.0f;
-                if (lane == 0) {
-                    const uint32_t target = (uint32_t)t.trows * (uint32_t)p.col_tiles;
-                    uint32_t spins = 0;
-                    uint32_t g = gave_up;
-                    while (!g && ld_acquire(done_ws + t.s) < target) {
-                        if (*(volatile uint32_t*)abort_flag != 0u) { g = 1u; break; }
-                        if (++spins > SPIN_LIMIT) {
-                            atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
-                            atomicExch(abort_flag, 1u);
-                            g = 1u;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    const float Ar = __uint_as_float(*(volatile const uint32_t*)(amax_row_ws + t.s));
-                    const float Ac = __uint_as_float(*(volatile const uint32_t*)(amax_col_ws + t.s));
-                    sr = global_encode(Ar);
-                    sc = global_encode(Ac);
-                    if (g) f |= H_GAVE_UP;
-                    // 0.25 folds into the column encode factor when neither 0.25 y
-                    // nor 0.25 enc can leave the normal range: A in [2^-100, 2^100]
-                    if (Ac >= 7.8886091e-31f && Ac <= 1.2676506e30f) f |= H_FOLD;
-                }
-                c_sr = __shfl_sync(0xFFFFFFFFu, sr, 0);
-                c_sc = __shfl_sync(0xFFFFFFFFu, sc, 0);
-                c_fl = __shfl_sync(0xFFFFFFFFu, f, 0);
-                gave_up = c_fl & H_GAVE_UP;
-                cached_s = t.s;
-            }
-            fl |= c_fl;
-            if (!(fl & H_GAVE_UP) && sh.tab_section[st] != t.s) {
-                // ---- this buffer's encode tables for section s (each lane
-                // writes and later reads only its own tab_section copy)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int code = lane + 32 * j;
-                    const bool z = code == 0 || code == 127;
-                    const float v = z ? 1.0f : e4m3_value((uint32_t)code);
-                    sh.enc_row[st][code] = z ? 0.0f : __fdiv_rn(c_sr, v);
-                    const float ec = z ? 0.0f : __fdiv_rn(c_sc, v);
-                    sh.enc_col[st][code] = (fl & H_FOLD) ? __fmul_rn(ec, 0.25f) : ec;
-                }
-                sh.tab_section[st] = t.s;
-            }
-        }
-        if (lane == 0) {
-            h.row0 = t.row0;
-            h.col0 = t.col0;
-            h.s = t.s;
-            h.r0s = t.r0s;
-            h.ms = t.ms;
-            h.row_in_sec0 = t.row_in_sec0;
-            h.flags = fl;
-            h.senc_r = c_sr;
-            h.senc_c = c_sc;
-        }
-        return fl;
-    }
+// ------------------------------------------------------ section records
+// A section's ready record (64 bits in the workspace, 0 until the section's
+// amax is complete) carries what its cast tiles need, so reading it is the
+// whole wait: low word senc_r | 1 << 31 (never 0 once written), high word
+// senc_c | fold << 31.  It is written by the compute warp whose amax tile
+// completes the section.
+__device__ __forceinline__ uint64_t* section_records(const NvParams& p) {
+    return reinterpret_cast<uint64_t*>(p.ws + ((NV_WS_HEADER + 3 * p.S + 1) & ~1));
 }
+__device__ __forceinline__ uint64_t make_record(float Ar, float Ac) {
+    // 0.25 folds into the column encode factor when neither 0.25 y nor
+    // 0.25 enc can leave the normal range: A in [2^-100, 2^100]
+    const uint32_t fold = (Ac >= 7.8886091e-31f && Ac <= 1.2676506e30f) ? 1u : 0u;
+    return (uint64_t)(__float_as_uint(global_encode(Ar)) | 0x80000000u) |
+           ((uint64_t)(__float_as_uint(global_encode(Ac)) | (fold << 31)) << 32);
+}
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* q) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(q) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* q, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(q), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* q, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(q), "r"(v) : "memory");
+    return old;
+}
+// Per-block encode factor S / value(sf), correctly rounded (0 for codes 0
+// and 127); `slow` when S is outside [2^-100, 2^100].
+__device__ __forceinline__ float block_enc(const NvShared& sh, uint32_t sf, float S, bool slow) {
+    const float2 vr = sh.vr[sf];
+    if (slow) return vr.x == 0.0f ? 0.0f : __fdiv_rn(S, vr.x);
+    return div_rn_neg(-S, Recip{vr.x, vr.y});
+}
+__device__ __forceinline__ bool slow_scale(float S) { return !(S >= 7.8886091e-31f && S <= 1.2676506e30f); }
 
 // ---------------------------------------------------------------- producer
+// Producer state that persists across buffer fills.
+struct ProducerState {
+    int seg = 0;                // schedule cursor
+    int ready_s = -1;           // section whose record is held below
+    uint32_t r_fl = 0;          // its header flags (H_FOLD, H_SLOW_*, H_GAVE_UP)
+    float r_sr = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
+    uint32_t gave_up = 0;       // sticky once a section wait gave up
+    int pf_s = -1;              // section of the prefetched record (lane 0)
+    uint64_t pf = 0;
+    TileInfo nt;                // the next fill's tile, decoded one fill ahead
+};
+
+// Header of buffer st for `tile` (and, for a cast tile, the section wait);
+// returns the header flags.
+__device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, const TileInfo& t, int lane,
+                                               ProducerState& ps) {
+    uint32_t* const err = p.ws + 2;
+    uint32_t* const abort_flag = p.ws + 3;
+    uint32_t fl = H_VALID;
+    if (t.phase == 1) {
+        fl |= H_CAST;
+        if (t.s != ps.ready_s) {
+            // ---- the section's record: prefetched one fill ahead, normally
+            // already written; else wait (bounded) for it
+            uint32_t f = 0u;
+            float sr = 1.0f, sc = 1.0f, scq = 1.0f;
+            if (lane == 0) {
+                const uint64_t* rec_ws = section_records(p) + t.s;
+                uint64_t rec = ps.pf_s == t.s ? ps.pf : ld_relaxed_u64(rec_ws);
+                uint32_t spins = 0;
+                uint32_t g = ps.gave_up;
+                while (!g && rec == 0u) {
+                    if (*(volatile uint32_t*)abort_flag != 0u) {
+                        g = 1u;
+                    } else if (++spins > SPIN_LIMIT) {
+                        atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
+                        atomicExch(abort_flag, 1u);
+                        g = 1u;
+                    } else {
+                        __nanosleep(64);
+                        rec = ld_relaxed_u64(rec_ws);
+                    }
+                }
+                if (g) {
+                    f |= H_GAVE_UP;
+                } else {
+                    sr = __uint_as_float((uint32_t)rec & 0x7FFFFFFFu);
+                    sc = __uint_as_float((uint32_t)(rec >> 32) & 0x7FFFFFFFu);
+                    scq = sc;
+                    if (rec >> 63) {
+                        f |= H_FOLD;
+                        scq = __fmul_rn(sc, 0.25f);  // exact: sc is in [2^-89, 2^111]
+                    }
+                    if (slow_scale(sr)) f |= H_SLOW_R;
+                    if (slow_scale(scq)) f |= H_SLOW_C;
+                }
+            }
+            ps.r_sr = __shfl_sync(0xFFFFFFFFu, sr, 0);
+            ps.r_sc = __shfl_sync(0xFFFFFFFFu, sc, 0);
+            ps.r_scq = __shfl_sync(0xFFFFFFFFu, scq, 0);
+            ps.r_fl = __shfl_sync(0xFFFFFFFFu, f, 0);
+            ps.gave_up = ps.r_fl & H_GAVE_UP;
+            ps.ready_s = t.s;
+        }
+        fl |= ps.r_fl;
+    }
+    if (lane == 0) {
+        StageHdr v;
+        v.row0 = t.row0;
+        v.col0 = t.col0;
+        v.s = t.s;
+        v.r0s = t.r0s;
+        v.ms = t.ms;
+        v.row_in_sec0 = t.row_in_sec0;
+        v.flags = fl;
+        v.senc_r = ps.r_sr;
+        v.senc_c = ps.r_sc;
+        v.senc_cq = ps.r_scq;
+        const uint4* src = reinterpret_cast<const uint4*>(&v);
+        uint4* dst = reinterpret_cast<uint4*>(&h);
+        dst[0] = src[0];
+        dst[1] = src[1];
+        dst[2] = src[2];
+    }
+    return fl;
+}
+
 // Returns the number of buffer fills started (the last one may be the
 // end-of-work header).
 __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh, uint32_t tiles_u32, int lane) {
@@ -263,20 +320,20 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
     uint32_t* const err = p.ws + 2;
     uint32_t* const abort_flag = p.ws + 3;
     const uint32_t total = p.total_items;
-    int seg = 0, cached_s = -1;
-    uint32_t c_fl = 0, gave_up = 0;
-    float c_sr = 1.0f, c_sc = 1.0f;
-    // Lane 0 keeps two claims in flight: fill k takes its tile from ca (k
-    // even) or cb (k odd) and refills that register with a new claim, read
-    // two fills later, so a claim's round trip overlaps two tile preparations.
-    uint32_t ca = 0, cb = 0;
+    ProducerState ps;
+    // Lane 0 keeps three claims in flight in ca, cb, cc: fill k takes its tile
+    // from one register, refills it with a new claim (read three fills
+    // later) and looks at the next fill's tile, claimed two fills earlier, to
+    // prefetch that tile's section record.
+    uint32_t ca = 0, cb = 0, cc = 0;
     if (lane == 0) {
         ca = atomicAdd(counter, 1u);
         cb = atomicAdd(counter, 1u);
+        cc = atomicAdd(counter, 1u);
     }
     uint32_t k = 0;
     // One buffer fill; false when the producer is done.
-    auto fill = [&](uint32_t& claim) -> bool {
+    auto fill = [&](uint32_t& claim, const uint32_t& next) -> bool {
         const int st = (int)(k % NST);
         StageHdr& h = sh.hdr[st];
         if (k >= NST && !mbar_wait_bounded(&sh.empty[st], ((k / NST) - 1u) & 1u, MBAR_LIMIT)) {
@@ -294,18 +351,28 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
             return false;
         }
         if (lane == 0) claim = atomicAdd(counter, 1u);
-        const uint32_t fl = nv_prepare(p, sh, h, st, tile, lane, seg, cached_s, c_fl, gave_up, c_sr, c_sc);
+        const TileInfo t = k == 1u ? decode(p, sh, tile, ps.seg) : ps.nt;
+        const uint32_t fl = nv_prepare(p, h, t, lane, ps);
         if (lane == 0 && !(fl & H_GAVE_UP)) {
             const uint32_t dst = tiles_u32 + (uint32_t)st * TILE_BYTES;
-            const int c1 = (int)(h.row0 / 16);
+            const int c1 = (int)(t.row0 / 16);
             mbar_expect_tx(&sh.full[st], (uint32_t)TILE_BYTES);
-            tma_load_3d(dst, &p.tmap, h.col0, c1, 0, &sh.full[st]);
-            tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, h.col0 + 64, c1, 0, &sh.full[st]);
+            tma_load_3d(dst, &p.tmap, t.col0, c1, 0, &sh.full[st]);
+            tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, t.col0 + 64, c1, 0, &sh.full[st]);
         }
-        mbar_arrive(&sh.full[st]);  // every lane: releases the header and table writes
+        mbar_arrive(&sh.full[st]);  // every lane: releases the header writes
+        // ---- prefetch the section record of the next fill's tile
+        const uint32_t nt = __shfl_sync(0xFFFFFFFFu, next, 0);
+        if (nt < total) {
+            ps.nt = decode(p, sh, nt, ps.seg);
+            if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s) {
+                ps.pf = ld_relaxed_u64(section_records(p) + ps.nt.s);
+                ps.pf_s = ps.nt.s;
+            }
+        }
         return true;
     };
-    while (fill(ca) && fill(cb)) {
+    while (fill(ca, cb) && fill(cb, cc) && fill(cc, ca)) {
     }
     return k;
 }
@@ -318,27 +385,38 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
     uint32_t* const amax_row_ws = p.ws + NV_WS_HEADER;
     uint32_t* const amax_col_ws = amax_row_ws + p.S;
     uint32_t* const done_ws = amax_col_ws + p.S;
-    const int64_t K = p.K;
     const bool do_row = p.flags & HQ_ROWWISE, do_col = p.flags & HQ_COLWISE;
 
     bf16_t sg[16];  // sigma_i as BF16 +-1
 #pragma unroll
     for (int i = 0; i < 16; ++i) sg[i] = ((p.sign_mask >> i) & 1u) ? (bf16_t)0xBF80u : (bf16_t)0x3F80u;
 
-    // rowwise: rows rr and rr + 4 (row block w / 2), 16-column block b =
-    // chunks 2b, 2b + 1; blocks 4..7 load the odd chunk first (swap = 1)
-    const int b = lane & 7;
-    const int rr = 8 * w + (lane >> 3);
-    const uint32_t swap = b >= 4 ? 1u : 0u;
-    const uint32_t re = chunk_off(b >> 2, rr >> 4, rr & 15, 2 * (b & 3));      // even chunk
-    const uint32_t ro = chunk_off(b >> 2, rr >> 4, rr & 15, 2 * (b & 3) + 1);  // odd chunk
-    const uint32_t r1 = swap ? ro : re;
-    const uint32_t roff[2] = {r1, r1 + 4u * 8u * 128u};  // row rr + 4: row in block + 4
-    const uint32_t roff2 = (swap ? re : ro) - r1;         // the other chunk, relative (mod 2^32)
-    // columnwise: BF16 pair 4w + jw (chunk w & 7 of half w >> 3), rows 16 rb + i
-    const int rb = lane & 7, jw = lane >> 3;
-    const uint32_t coff = chunk_off(w >> 3, rb, 0, w & 7) + 4u * (uint32_t)jw;
-    const int cpair = 8 * w + 2 * jw;  // first of the two columns, inside the tile
+    const int b = lane & 7;                  // rowwise 16-column block
+    const int rb = lane & 7, jw = lane >> 3;  // columnwise 16-row block, BF16 pair in the chunk
+    const uint32_t swap = b >= 4 ? 1u : 0u;  // blocks 4..7 load their odd chunk first
+    const uint64_t K2 = (uint64_t)p.K / 2, K16 = (uint64_t)p.K / 16;
+    // The 16 parts of a tile (see the header) are shared out among the NCW
+    // compute warps: warp w takes parts w, w + NCW, ...  Per part, this lane's
+    // shared offsets and output offsets:
+    struct Part {
+        uint32_t roff0;    // rowwise: first chunk of row rr (row rr + 4: + 4096)
+        uint32_t roff2;    //   the other chunk, relative (mod 2^32)
+        uint32_t coff;     // columnwise: pair 4 vw + jw, row 16 rb
+        int cpair;         //   first of its two columns, inside the tile
+        uint64_t rs_off0;  // row rr's block-scale offset (+ 4 K16 for rr + 4; codes at 8x)
+    };
+    auto part = [&](int vw) {
+        Part q;
+        const int rr = 8 * vw + (lane >> 3);  // rows rr, rr + 4 in row block vw / 2
+        const uint32_t re = chunk_off(b >> 2, rr >> 4, rr & 15, 2 * (b & 3));      // even chunk
+        const uint32_t ro = chunk_off(b >> 2, rr >> 4, rr & 15, 2 * (b & 3) + 1);  // odd chunk
+        q.roff0 = swap ? ro : re;
+        q.roff2 = (swap ? re : ro) - q.roff0;
+        q.coff = chunk_off(vw >> 3, rb, 0, vw & 7) + 4u * (uint32_t)jw;  // chunk vw & 7 of half vw >> 3
+        q.cpair = 8 * vw + 2 * jw;
+        q.rs_off0 = (uint64_t)rr * K16 + b;
+        return q;
+    };
 
     for (uint32_t k = 0;; ++k) {
         const int st = (int)(k % NST);
@@ -349,7 +427,14 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             }
             break;
         }
-        const StageHdr h = sh.hdr[st];
+        StageHdr h;
+        {
+            const uint4* src = reinterpret_cast<const uint4*>(&sh.hdr[st]);
+            uint4* dst = reinterpret_cast<uint4*>(&h);
+            dst[0] = src[0];
+            dst[1] = src[1];
+            dst[2] = src[2];
+        }
         if (!(h.flags & H_VALID)) break;
         const uint8_t* T = tiles + (size_t)st * TILE_BYTES;
 
@@ -357,11 +442,14 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             // ===================================================== amax tile
             uint32_t mrow = 0u;
             float mcol = 0.0f;
+            for (int vw = w; vw < 16; vw += NCW) {
+            const Part pt = part(vw);
             if (do_row) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
-                    const uint4 lo = *reinterpret_cast<const uint4*>(T + roff[kk]);  // (odd chunk if swap)
-                    const uint4 hi = *reinterpret_cast<const uint4*>(T + (roff[kk] + roff2));
+                    const uint32_t ro = pt.roff0 + 4096u * kk;
+                    const uint4 lo = *reinterpret_cast<const uint4*>(T + ro);  // (odd chunk if swap)
+                    const uint4 hi = *reinterpret_cast<const uint4*>(T + (ro + pt.roff2));
                     const uint32_t m = hmax_abs(hmax_abs(hmax_abs(lo.x, lo.y), hmax_abs(lo.z, lo.w)),
                                                 hmax_abs(hmax_abs(hi.x, hi.y), hmax_abs(hi.z, hi.w)));
                     mrow = max(mrow, halves_max_bits(m));
@@ -370,7 +458,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             if (do_col) {
                 uint32_t x[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + coff + 1024 * i);
+                for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + pt.coff + 1024 * i);
                 f2 v[16];
                 column_rht(x, sg, v);
 #pragma unroll
@@ -380,6 +468,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     mcol = absmax3(mcol, a0, a1);
                 }
             }
+            }  // parts
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) {
                 mrow = max(mrow, __shfl_xor_sync(0xFFFFFFFFu, mrow, o));
@@ -400,22 +489,34 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     sh.acc_cnt[st] = 0u;
                     if (do_row) atomicMax(amax_row_ws + h.s, ar);
                     if (do_col) atomicMax(amax_col_ws + h.s, ac);
-                    red_release_add(done_ws + h.s, 1u);  // release: the maxima above are visible first
+                    // acq_rel: the maxima above are visible first, and the
+                    // tile completing the section sees every tile's maxima
+                    const uint32_t target = (uint32_t)(h.ms / NV_TILE) * (uint32_t)p.col_tiles;
+                    if (atom_add_acq_rel(done_ws + h.s, 1u) == target - 1u) {
+                        const float Ar = __uint_as_float(*(volatile uint32_t*)(amax_row_ws + h.s));
+                        const float Ac = __uint_as_float(*(volatile uint32_t*)(amax_col_ws + h.s));
+                        st_relaxed_u64(section_records(p) + h.s, make_record(Ar, Ac));
+                    }
                 }
             }
         } else if (!(h.flags & H_GAVE_UP)) {
             // ===================================================== cast tile
+            uint8_t* const rc_base = p.row_codes + (uint64_t)h.row0 * K2 + (uint32_t)h.col0 / 2u;
+            uint8_t* const rs_base = p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
+            for (int vw = w; vw < 16; vw += NCW) {
+            const Part pt = part(vw);
             if (do_row) {
-                const float* enc_tab = sh.enc_row[st];
+                const bool slow = h.flags & H_SLOW_R;
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
-                    const uint4 lo = *reinterpret_cast<const uint4*>(T + roff[kk]);  // (odd chunk if swap)
-                    const uint4 hi = *reinterpret_cast<const uint4*>(T + (roff[kk] + roff2));
+                    const uint32_t ro = pt.roff0 + 4096u * kk;
+                    const uint4 lo = *reinterpret_cast<const uint4*>(T + ro);  // (odd chunk if swap)
+                    const uint4 hi = *reinterpret_cast<const uint4*>(T + (ro + pt.roff2));
                     const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
                     const uint32_t m = hmax_abs(hmax_abs(hmax_abs(wd[0], wd[1]), hmax_abs(wd[2], wd[3])),
                                                 hmax_abs(hmax_abs(wd[4], wd[5]), hmax_abs(wd[6], wd[7])));
                     const uint32_t sf = block_sf(__uint_as_float(halves_max_bits(m)), h.senc_r);
-                    const float enc = enc_tab[sf];
+                    const float enc = block_enc(sh, sf, h.senc_r, slow);
                     const f2 e2 = pack2(enc, enc);
                     float q[16];
 #pragma unroll
@@ -424,19 +525,18 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                         split_bf16x2(wd[c], xl, xh);
                         unpack2(mul2(pack2(add_bf16(xl, -0.0f), add_bf16(xh, -0.0f)), e2), q[2 * c], q[2 * c + 1]);
                     }
-                    const int64_t row = h.row0 + rr + 4 * kk;
-                    const int64_t col = h.col0 + 16 * b;
                     const uint32_t c0 = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
                     const uint32_t c1 = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-                    *reinterpret_cast<uint2*>(p.row_codes + row * (K / 2) + col / 2) =
+                    const uint64_t rs_off = pt.rs_off0 + (kk ? 4u * K16 : 0u);
+                    *reinterpret_cast<uint2*>(rc_base + 8u * rs_off) =
                         swap ? make_uint2(c1, c0) : make_uint2(c0, c1);
-                    p.row_sf[row * (K / 16) + col / 16] = (uint8_t)sf;
+                    rs_base[rs_off] = (uint8_t)sf;
                 }
             }
             if (do_col) {
                 uint32_t x[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + coff + 1024 * i);
+                for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + pt.coff + 1024 * i);
                 f2 v[16];
                 column_rht(x, sg, v);
                 float a0 = 0.0f, a1 = 0.0f;
@@ -450,7 +550,8 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 }
                 const uint32_t sf0 = block_sf(__fmul_rn(a0, 0.25f), h.senc_c);
                 const uint32_t sf1 = block_sf(__fmul_rn(a1, 0.25f), h.senc_c);
-                const f2 e2 = pack2(sh.enc_col[st][sf0], sh.enc_col[st][sf1]);
+                const bool slow = h.flags & H_SLOW_C;
+                const f2 e2 = pack2(block_enc(sh, sf0, h.senc_cq, slow), block_enc(sh, sf1, h.senc_cq, slow));
                 if (!(h.flags & H_FOLD)) {
                     const f2 quarter = pack2(0.25f, 0.25f);
 #pragma unroll
@@ -459,19 +560,23 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 float q0[16], q1[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) unpack2(mul2(v[i], e2), q0[i], q1[i]);
-                const int64_t ms = h.ms;
-                const int64_t c = h.col0 + cpair;
-                uint8_t* cb = p.col_codes + K * (int64_t)h.r0s / 2 + (h.row_in_sec0 + 16 * rb) / 2;
-                uint8_t* sb = p.col_sf + K * (int64_t)h.r0s / 16 + (h.row_in_sec0 / 16 + rb);
-                *reinterpret_cast<uint2*>(cb + c * (ms / 2)) =
+                // transposed section block: column c of the section at c * ms / 2
+                const uint32_t ms2 = (uint32_t)h.ms / 2u, ms16 = (uint32_t)h.ms / 16u;
+                const uint64_t c = (uint32_t)(h.col0 + pt.cpair);
+                uint8_t* const cb = p.col_codes + (uint64_t)h.r0s * K2 + c * ms2 +
+                                    ((uint32_t)h.row_in_sec0 / 2u + 8u * (uint32_t)rb);
+                uint8_t* const sb = p.col_sf + (uint64_t)h.r0s * K16 + c * ms16 +
+                                    ((uint32_t)h.row_in_sec0 / 16u + (uint32_t)rb);
+                *reinterpret_cast<uint2*>(cb) =
                     make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
                                e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
-                *reinterpret_cast<uint2*>(cb + (c + 1) * (ms / 2)) =
+                *reinterpret_cast<uint2*>(cb + ms2) =
                     make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
                                e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
-                sb[c * (ms / 16)] = (uint8_t)sf0;
-                sb[(c + 1) * (ms / 16)] = (uint8_t)sf1;
+                sb[0] = (uint8_t)sf0;
+                sb[ms16] = (uint8_t)sf1;
             }
+            }  // parts
         }
         mbar_arrive(&sh.empty[st]);  // every compute thread: this thread is done with the buffer
     }
@@ -479,7 +584,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
 }  // namespace
 
-__global__ void __launch_bounds__(NV_THREADS, 1) nvfp4_group_kernel(const __grid_constant__ NvParams p) {
+__global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel(const __grid_constant__ NvParams p) {
     extern __shared__ __align__(1024) uint8_t nv_smem_raw[];
     uint8_t* const nv_smem = nv_smem_raw + ((1024u - (smem_u32(nv_smem_raw) & 1023u)) & 1023u);
     NvShared& sh = *reinterpret_cast<NvShared*>(nv_smem + NST * TILE_BYTES);
@@ -499,13 +604,21 @@ __global__ void __launch_bounds__(NV_THREADS, 1) nvfp4_group_kernel(const __grid
             sh.acc_row[st] = 0u;
             sh.acc_col[st] = 0u;
             sh.acc_cnt[st] = 0u;
-            sh.tab_section[st] = -1;
         }
         fence_mbar_init();
     }
     for (int i = tid; i <= p.nseg; i += NV_THREADS) sh.seg_start[i] = p.seg_start[i];
     for (int i = tid; i < p.nseg; i += NV_THREADS) sh.seg_info[i] = p.seg_info[i];
     for (int i = tid; i <= p.S; i += NV_THREADS) sh.sec_row0[i] = p.sec_row0[i];
+    for (int i = tid; i < p.S; i += NV_THREADS) {
+        const uint32_t trows = (uint32_t)(p.sec_row0[i + 1] - p.sec_row0[i]) / NV_TILE;
+        sh.sec_magic[i] = trows ? 0xFFFFFFFFu / trows : 0u;
+    }
+    if (tid < 128) {
+        const bool z = tid == 0 || tid == 127;
+        const float v = z ? 0.0f : e4m3_value((uint32_t)tid);
+        sh.vr[tid] = make_float2(v, z ? -0.0f : -__frcp_rn(v));
+    }
     __syncthreads();
     if (warp == NCW) {
         const uint32_t fills = nv_producer(p, sh, smem_u32(nv_smem), lane);
@@ -545,6 +658,7 @@ __global__ void __launch_bounds__(NV_THREADS, 1) nvfp4_group_kernel(const __grid
                 amax_col_ws[s] = 0;
             }
             done_ws[s] = 0;
+            section_records(p)[s] = 0u;
         }
     }
     if (tid == 0 && p.reset_counter) {
@@ -561,7 +675,7 @@ int nvfp4_blocks_per_sm() {
     return n > 0 ? n : 1;
 }
 
-int nvfp4_tiles_in_flight_per_cta() { return NST + 2; }
+int nvfp4_tiles_in_flight_per_cta() { return NST + 3; }
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
     nvfp4_group_kernel<<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
