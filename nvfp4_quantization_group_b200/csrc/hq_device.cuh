@@ -98,42 +98,6 @@ __device__ __forceinline__ float absmax3(float m, float a, float b) {
     return r;
 }
 
-// ------------------------------------------------------------ Hadamard
-// Unnormalised Sylvester butterfly, stages h = 1, 2, 4, ... ascending:
-// (a, b) -> (a + b, a - b) for every pair (i, i + h) with (i & h) == 0.
-
-// In place on N scalars held in registers (N a power of two).
-template <int N>
-__device__ __forceinline__ void fwht_regs(float (&v)[N]) {
-#pragma unroll
-    for (int h = 1; h < N; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-            if ((i & h) == 0) {
-                float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
-            }
-        }
-    }
-}
-
-// The same butterfly over index i of 16 packed pairs: pair i holds element i
-// of two independent vectors, so both transforms run in one f32x2 op each.
-__device__ __forceinline__ void fwht16_x2(f2 (&v)[16]) {
-#pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            if ((i & h) == 0) {
-                f2 a = v[i], b = v[i + h];
-                v[i] = add2(a, b);
-                v[i + h] = sub2(a, b);
-            }
-        }
-    }
-}
-
 // -------------------------------------------------------------- FP8 rule
 // Scale of one group: max(amax, 1e-10f) * float32(1/448).
 __device__ __forceinline__ float fp8_group_scale(float amax) {
@@ -196,31 +160,6 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint4 ld_nc_v4_hint(const void* p, uint64_t policy) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p), "l"(policy));
-    return v;
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
-}
-
 }  // namespace hq
 
 namespace hq {
@@ -259,19 +198,8 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" :: "r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
-                 :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-// true once the phase with parity `parity` of the barrier has completed
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-// As mbar_try_wait, but the thread sleeps until the phase completes or about
-// `ns` nanoseconds pass (no polling traffic while it waits).
+// true once the phase with parity `parity` of the barrier has completed; the
+// thread sleeps until then or until about `ns` nanoseconds pass.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -298,27 +226,4 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int 
                  " [%0], [%1, {%2, %3, %4}], [%5];"
                  :: "r"(dst), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(threads) : "memory");
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
-
-// 16-byte asynchronous copy global -> shared (cp.async, L1 bypassed), and
-// its group commit / wait.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
-}
-// Arrive on `bar` once every cp.async this thread issued so far has landed
-// (the arrival is counted in the barrier's initial count: .noinc).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 }  // namespace hq
