@@ -269,13 +269,15 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     p.a_width = a_width;
     p.b_width = b_width;
     p.nvec = M * G;
+    p.M = M;
     p.G = G;
     p.rotate = hadamard_n == 128;
     p.out = out_fp8;
     p.scales = scales;
     p.scale_layout = scale_layout;
     p.scale_ld = scale_ld;
-    const int64_t tiles = (p.nvec + 127) / 128;
+    p.ntiles = cat_rotate_tiles(p);
+    const int64_t tiles = p.ntiles;
     const int64_t cap = (int64_t)dev->sms * (dev->cat_blocks_per_sm > 0 ? dev->cat_blocks_per_sm : 1);
     const int grid = (int)(tiles < cap ? tiles : cap);
     launch_cat_rotate(p, grid, (cudaStream_t)stream);

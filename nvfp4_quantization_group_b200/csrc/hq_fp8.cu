@@ -54,122 +54,179 @@ __device__ __forceinline__ uint2 quant8(const f2 (&ny)[4], float s) {
 }
 
 // ------------------------------------------------ cat -> H128 -> FP8 1x128
-// One thread owns one 128-vector per tile.  A tile of 128 vectors is staged
-// through shared memory twice: the BF16 inputs arrive with coalesced 16-byte
-// loads (16 consecutive threads read one vector's 256 bytes) and are read
-// back one vector per thread; the codes go out the same way in reverse.
-// 16-byte chunk c of vector v sits at slot v * W + (c ^ (v & 7)), which keeps
-// both access patterns free of shared-memory bank conflicts.
-constexpr int CAT_THREADS = 128;
+// Eight threads share one 128-vector, 16 elements each; a CTA of 256 threads
+// takes a tile of 32 vectors.  The butterfly runs in two halves:
+//  * thread j loads elements 16j..16j+15 (two 16-byte loads, from the pe or
+//    the nope part) and runs stages 1, 2, 4, 8 on them; stage 1 takes the
+//    BF16 pair straight from the load word (mixed-precision add / FMA, one
+//    rounding each, as FP32 additions of the widened values);
+//  * the 8 threads exchange values through shared memory (within the warp,
+//    no CTA barrier) so that thread j then holds elements 16s + 2j and
+//    16s + 2j + 1 for s = 0..7, and runs stages 16, 32, 64 on them.
+// The 8 threads then reduce the amax with 3 shuffles, quantize their 16
+// values, and exchange the codes through shared memory once more so that
+// each writes 16 contiguous bytes.  Tiles are 32 consecutive vectors, or, for
+// transposed scales, 32 consecutive rows of one group (the 32 scales are then
+// contiguous).  The next tile's loads are issued before the current tile is
+// computed.
+constexpr int CAT_THREADS = 256;
+constexpr int CAT_VEC = 32;  // vectors per tile
 
-__global__ void __launch_bounds__(CAT_THREADS, 2) cat_rotate_fp8_kernel(CatRotateParams p) {
-    __shared__ __align__(16) uint4 stage[CAT_THREADS * 16];  // 32 KB
-    const int tid = threadIdx.x;
+struct CatShared {
+    float2 t[CAT_VEC][72];       // 64 pairs of one vector + 8 of padding (bank spread)
+    uint32_t codes[CAT_VEC][36];  // 128 code bytes of one vector + 16 of padding
+};
+
+// Vector index of slot k (0..31) of tile `tile`, or -1 past the end.
+__device__ __forceinline__ int64_t cat_vector(const CatRotateParams& p, int64_t tile, int k) {
+    if (p.scale_layout == 0) {
+        const int64_t v = tile * CAT_VEC + k;
+        return v < p.nvec ? v : -1;
+    }
+    const int64_t row_tiles = (p.M + CAT_VEC - 1) / CAT_VEC;
+    const int64_t g = tile / row_tiles;
+    const int64_t t = (tile - g * row_tiles) * CAT_VEC + k;
+    return t < p.M ? t * p.G + g : -1;
+}
+
+// The two 16-byte chunks (elements 16j..16j+15) of vector v.
+__device__ __forceinline__ void cat_load(const CatRotateParams& p, int64_t v, int j, uint4& c0, uint4& c1) {
+    c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+    if (v < 0) return;
+    const int64_t t = v / p.G;
+    const int g = (int)(v - t * p.G);
     const int a_chunks = p.a_width / 8;
-    const int64_t ntiles = (p.nvec + CAT_THREADS - 1) / CAT_THREADS;
-    // -1 / sqrt(128): the negated numerators feed the division directly
-    const float neg_c128 = -__uint_as_float(0x3DB504F3u);
-
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        const int64_t v0 = tile * CAT_THREADS;
-        // ---- coalesced load of 128 vectors x 16 chunks
-#pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-            const int q = it * CAT_THREADS + tid;
-            const int vv = q >> 4, c = q & 15;
-            const int64_t v = v0 + vv;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (v < p.nvec) {
-                const int64_t t = v / p.G;
-                const int g = (int)(v - t * p.G);
-                const uint16_t* src = c < a_chunks
-                    ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + c * 8
-                    : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (c - a_chunks) * 8;
-                val = ld_nc_v4(src);
-            }
-            stage[vv * 16 + (c ^ (vv & 7))] = val;
-        }
-        __syncthreads();
-
-        // ---- own vector: BF16 -> FP32, negated (the quantizer takes -y)
-        float y[128];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            uint4 w = stage[tid * 16 + (c ^ (tid & 7))];
-            y[8 * c + 0] = bf16_lo(w.x); y[8 * c + 1] = bf16_hi(w.x);
-            y[8 * c + 2] = bf16_lo(w.y); y[8 * c + 3] = bf16_hi(w.y);
-            y[8 * c + 4] = bf16_lo(w.z); y[8 * c + 5] = bf16_hi(w.z);
-            y[8 * c + 6] = bf16_lo(w.w); y[8 * c + 7] = bf16_hi(w.w);
-        }
-        __syncthreads();  // the staging buffer is reused for the codes
+    for (int h = 0; h < 2; ++h) {
+        const int c = 2 * j + h;
+        const uint16_t* src = c < a_chunks
+            ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + c * 8
+            : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (c - a_chunks) * 8;
+        (h ? c1 : c0) = ld_nc_v4(src);
+    }
+}
 
+__global__ void __launch_bounds__(CAT_THREADS, 3) cat_rotate_fp8_kernel(CatRotateParams p) {
+    __shared__ CatShared sh;
+    const int tid = threadIdx.x, k = tid >> 3, j = tid & 7;
+    const float neg_c128 = -__uint_as_float(0x3DB504F3u);  // -RN(1/sqrt(128)): negated numerators
+    const bf16_t minus_one = (bf16_t)0xBF80u;
+
+    int64_t tile = blockIdx.x;
+    uint4 n0, n1;  // the next tile's chunks
+    cat_load(p, tile < p.ntiles ? cat_vector(p, tile, k) : -1, j, n0, n1);
+    for (; tile < p.ntiles; tile += gridDim.x) {
+        const int64_t v = cat_vector(p, tile, k);
+        const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+        const int64_t nt = tile + gridDim.x;
+        cat_load(p, nt < p.ntiles ? cat_vector(p, nt, k) : -1, j, n0, n1);
+
+        // ---- elements 16j..16j+15 as 8 pairs (2i, 2i+1) of this segment
+        f2 y[8];
         if (p.rotate) {
-            // Sylvester butterfly, stages 1, 2, ..., 64 (ascending), then
-            // the orthonormal scale; stage 1 is scalar, the rest packed.
 #pragma unroll
-            for (int i = 0; i < 128; i += 2) {
-                float a = y[i], b = y[i + 1];
-                y[i] = __fadd_rn(a, b);
-                y[i + 1] = __fsub_rn(a, b);
+            for (int i = 0; i < 8; ++i) {
+                bf16_t lo, hi;
+                split_bf16x2(w[i], lo, hi);
+                const float x0 = bf16_lo(w[i]);
+                y[i] = pack2(add_bf16(hi, x0), fma_bf16(hi, minus_one, x0));  // stage 1
             }
-            f2 v2[64];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v2[i] = pack2(y[2 * i], y[2 * i + 1]);
+            for (int h = 1; h < 8; h <<= 1) {  // stages 2, 4, 8
 #pragma unroll
-            for (int h = 1; h < 64; h <<= 1) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     if ((i & h) == 0) {
-                        f2 a = v2[i], b = v2[i + h];
-                        v2[i] = add2(a, b);
-                        v2[i + h] = sub2(a, b);
+                        const f2 a = y[i], b = y[i + h];
+                        y[i] = add2(a, b);
+                        y[i + h] = sub2(a, b);
                     }
                 }
             }
-            const f2 nc2 = pack2(neg_c128, neg_c128);
-#pragma unroll
-            for (int i = 0; i < 64; ++i) unpack2(mul2(v2[i], nc2), y[2 * i], y[2 * i + 1]);
         } else {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) y[i] = -y[i];
+            for (int i = 0; i < 8; ++i) y[i] = pack2(bf16_lo(w[i]), bf16_hi(w[i]));
         }
-
-        // ---- group scale and codes
+        // ---- exchange: thread j now takes pair j of every segment s
+        // (16-byte piece c of segment s is stored at position (c + s/2) & 3 of
+        // the segment's 64 bytes: the 8 lanes of a vector then hit 8
+        // different bank groups when writing)
+        float4* row = reinterpret_cast<float4*>(&sh.t[k][8 * j]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float a0, a1, b0, b1;
+            unpack2(y[2 * c], a0, a1);
+            unpack2(y[2 * c + 1], b0, b1);
+            row[(c + (j >> 1)) & 3] = make_float4(a0, a1, b0, b1);
+        }
+        __syncwarp();
+        f2 z[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const float2 e = sh.t[k][8 * s + 2 * (((j >> 1) + (s >> 1)) & 3) + (j & 1)];
+            z[s] = pack2(e.x, e.y);
+        }
+        if (p.rotate) {
+#pragma unroll
+            for (int h = 1; h < 8; h <<= 1) {  // stages 16, 32, 64
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    if ((s & h) == 0) {
+                        const f2 a = z[s], b = z[s + h];
+                        z[s] = add2(a, b);
+                        z[s + h] = sub2(a, b);
+                    }
+                }
+            }
+        }
+        const f2 nc2 = pack2(p.rotate ? neg_c128 : -1.0f, p.rotate ? neg_c128 : -1.0f);
         float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 128; i += 2) amax = absmax3(amax, y[i], y[i + 1]);
-        const float s = fp8_group_scale(amax);
+        for (int s = 0; s < 8; ++s) {
+            z[s] = mul2(z[s], nc2);  // -y (exact negation when not rotating)
+            float a, b;
+            unpack2(z[s], a, b);
+            amax = absmax3(amax, a, b);
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+        const float sc = fp8_group_scale(amax);
+        // ---- codes of elements 16s + 2j, 16s + 2j + 1
+        uint32_t q[8];
+        if (!isinf(sc)) {
+            const Recip d = make_recip(sc);
+            const f2 b2 = pack2(d.b, d.b), nr2 = pack2(d.nr, d.nr);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            f2 a[4], b[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[i] = pack2(y[16 * c + 2 * i], y[16 * c + 2 * i + 1]);
-                b[i] = pack2(y[16 * c + 8 + 2 * i], y[16 * c + 8 + 2 * i + 1]);
+            for (int s = 0; s < 8; ++s) {
+                float a, b;
+                unpack2(div2_rn_neg(z[s], b2, nr2), a, b);
+                q[s] = e4m3x2(a, b);
             }
-            uint2 lo = quant8(a, s), hi = quant8(b, s);
-            stage[tid * 8 + (c ^ (tid & 7))] = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        }
-        const int64_t v = v0 + tid;
-        if (v < p.nvec) {
-            if (p.scale_layout == 0) {
-                p.scales[v] = s;
-            } else {
-                const int64_t t = v / p.G;
-                const int g = (int)(v - t * p.G);
-                p.scales[(int64_t)g * p.scale_ld + t] = s;
+        } else {  // an infinite input: plain IEEE division
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                float a, b;
+                unpack2(z[s], a, b);
+                q[s] = e4m3x2(__fdiv_rn(-a, sc), __fdiv_rn(-b, sc));
             }
         }
-        __syncthreads();
-        // ---- coalesced store of 128 vectors x 8 chunks of codes
-        uint4* out = reinterpret_cast<uint4*>(p.out) + v0 * 8;
+        uint16_t* cb = reinterpret_cast<uint16_t*>(sh.codes[k]);
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-            const int q = it * CAT_THREADS + tid;
-            const int vv = q >> 3, c = q & 7;
-            if (v0 + vv < p.nvec) out[q] = stage[vv * 8 + (c ^ (vv & 7))];
+        for (int s = 0; s < 8; ++s) cb[8 * s + j] = (uint16_t)q[s];
+        __syncwarp();
+        if (v >= 0) {
+            const uint4 out = *reinterpret_cast<const uint4*>(&sh.codes[k][4 * j]);
+            *reinterpret_cast<uint4*>(p.out + v * 128 + 16 * j) = out;
+            if (j == 0) {
+                if (p.scale_layout == 0) {
+                    p.scales[v] = sc;
+                } else {
+                    const int64_t t = v / p.G;
+                    p.scales[(v - t * p.G) * p.scale_ld + t] = sc;
+                }
+            }
         }
-        __syncthreads();
+        __syncwarp();  // the exchange buffers are reused by the next tile
     }
 }
 
@@ -265,6 +322,10 @@ __global__ void convert_kernel(int fmt, const float* in, uint8_t* out, int64_t n
 }
 
 // ------------------------------------------------------------ launchers
+int64_t cat_rotate_tiles(const CatRotateParams& p) {
+    return p.scale_layout == 0 ? (p.nvec + CAT_VEC - 1) / CAT_VEC : p.G * ((p.M + CAT_VEC - 1) / CAT_VEC);
+}
+
 int cat_rotate_blocks_per_sm() {
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cat_rotate_fp8_kernel, CAT_THREADS, 0);

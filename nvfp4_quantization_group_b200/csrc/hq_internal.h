@@ -18,6 +18,8 @@ struct CatRotateParams {
     int64_t a_row_stride, b_row_stride;
     int a_width, b_width;
     int64_t nvec;  // M * G vectors of 128
+    int64_t M;     // rows (tokens)
+    int64_t ntiles;  // tiles of 32 vectors (see cat_rotate_tiles)
     int G;
     int rotate;    // 1: H128 / sqrt(128); 0: none
     uint8_t* out;
@@ -38,6 +40,7 @@ constexpr int K128_THREADS = 256;   // 8 warps, two K128 groups per warp step
 constexpr int K128_UNROLL = 4;      // warp steps with loads in flight
 
 int cat_rotate_blocks_per_sm();
+int64_t cat_rotate_tiles(const CatRotateParams& p);
 void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st);
 void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st);
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st);
