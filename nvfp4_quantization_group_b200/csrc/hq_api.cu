@@ -277,6 +277,9 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     p.scale_layout = scale_layout;
     p.scale_ld = scale_ld;
     p.ntiles = cat_rotate_tiles(p);
+    if (p.nvec >= ((int64_t)1 << 31) || p.ntiles >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
+    p.g_magic = 0xFFFFFFFFu / (uint32_t)G;
+    p.gt_magic = 0xFFFFFFFFu / (uint32_t)cat_rotate_group_tiles(G);
     const int64_t tiles = p.ntiles;
     const int64_t cap = (int64_t)dev->sms * (dev->cat_blocks_per_sm > 0 ? dev->cat_blocks_per_sm : 1);
     const int grid = (int)(tiles < cap ? tiles : cap);

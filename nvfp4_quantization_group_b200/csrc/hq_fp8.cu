@@ -77,24 +77,59 @@ struct CatShared {
     uint32_t codes[CAT_VEC][36];  // 128 code bytes of one vector + 16 of padding
 };
 
-// Vector index of slot k (0..31) of tile `tile`, or -1 past the end.
-__device__ __forceinline__ int64_t cat_vector(const CatRotateParams& p, int64_t tile, int k) {
-    if (p.scale_layout == 0) {
-        const int64_t v = tile * CAT_VEC + k;
-        return v < p.nvec ? v : -1;
+#ifndef HQ_CAT_TT
+#define HQ_CAT_TT 8
+#endif
+#ifndef HQ_CAT_MINB
+#define HQ_CAT_MINB 3
+#endif
+// Transposed scales: a tile is CAT_TT consecutive rows x CAT_TG groups, slot
+// k = (k / CAT_TT) groups on, (k % CAT_TT) rows on, so each group's CAT_TT
+// scales are contiguous; consecutive tiles walk the groups of a row block.
+constexpr int CAT_TT = HQ_CAT_TT, CAT_TG = CAT_VEC / CAT_TT;
+
+// x / d and x % d for 32-bit x by multiply-high with m = floor((2^32 - 1) / d)
+// and at most two corrections.
+__device__ __forceinline__ uint32_t udivmod(uint32_t x, uint32_t d, uint32_t m, uint32_t& r) {
+    uint32_t q = __umulhi(x, m);
+    r = x - q * d;
+    while (r >= d) {
+        ++q;
+        r -= d;
     }
-    const int64_t row_tiles = (p.M + CAT_VEC - 1) / CAT_VEC;
-    const int64_t g = tile / row_tiles;
-    const int64_t t = (tile - g * row_tiles) * CAT_VEC + k;
-    return t < p.M ? t * p.G + g : -1;
+    return q;
 }
 
-// The two 16-byte chunks (elements 16j..16j+15) of vector v.
-__device__ __forceinline__ void cat_load(const CatRotateParams& p, int64_t v, int j, uint4& c0, uint4& c1) {
+struct CatVec {
+    int t, g;  // row and group; t < 0 past the end
+};
+
+// Row and group of slot k (0..31) of tile `tile` (host: tiles, vectors < 2^31).
+__device__ __forceinline__ CatVec cat_vector(const CatRotateParams& p, uint32_t tile, int k) {
+    CatVec r;
+    if (p.scale_layout == 0) {
+        const uint32_t v = tile * CAT_VEC + k;
+        uint32_t g;
+        r.t = (int)udivmod(v, (uint32_t)p.G, p.g_magic, g);
+        r.g = (int)g;
+        if ((int64_t)v >= p.nvec) r.t = -1;
+        return r;
+    }
+    const uint32_t g_tiles = ((uint32_t)p.G + CAT_TG - 1) / CAT_TG;
+    uint32_t gb;
+    const uint32_t tb = udivmod(tile, g_tiles, p.gt_magic, gb);
+    r.g = (int)(gb * CAT_TG) + k / CAT_TT;
+    r.t = (int)(tb * CAT_TT) + k % CAT_TT;
+    if (r.t >= p.M || r.g >= p.G) r.t = -1;
+    return r;
+}
+
+// The two 16-byte chunks (elements 16j..16j+15) of vector (t, g).
+__device__ __forceinline__ void cat_load(const CatRotateParams& p, CatVec cv, int j, uint4& c0, uint4& c1) {
     c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
-    if (v < 0) return;
-    const int64_t t = v / p.G;
-    const int g = (int)(v - t * p.G);
+    if (cv.t < 0) return;
+    const int64_t t = cv.t;
+    const int g = cv.g;
     const int a_chunks = p.a_width / 8;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -106,20 +141,24 @@ __device__ __forceinline__ void cat_load(const CatRotateParams& p, int64_t v, in
     }
 }
 
-__global__ void __launch_bounds__(CAT_THREADS, 3) cat_rotate_fp8_kernel(CatRotateParams p) {
+__global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_fp8_kernel(CatRotateParams p) {
     __shared__ CatShared sh;
     const int tid = threadIdx.x, k = tid >> 3, j = tid & 7;
     const float neg_c128 = -__uint_as_float(0x3DB504F3u);  // -RN(1/sqrt(128)): negated numerators
     const bf16_t minus_one = (bf16_t)0xBF80u;
 
-    int64_t tile = blockIdx.x;
+    const CatVec none{-1, 0};
+    uint32_t tile = blockIdx.x;
+    const uint32_t ntiles = (uint32_t)p.ntiles;
     uint4 n0, n1;  // the next tile's chunks
-    cat_load(p, tile < p.ntiles ? cat_vector(p, tile, k) : -1, j, n0, n1);
-    for (; tile < p.ntiles; tile += gridDim.x) {
-        const int64_t v = cat_vector(p, tile, k);
+    CatVec nv = tile < ntiles ? cat_vector(p, tile, k) : none;
+    cat_load(p, nv, j, n0, n1);
+    for (; tile < ntiles; tile += gridDim.x) {
+        const CatVec cv = nv;
         const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-        const int64_t nt = tile + gridDim.x;
-        cat_load(p, nt < p.ntiles ? cat_vector(p, nt, k) : -1, j, n0, n1);
+        const uint32_t nt = tile + gridDim.x;
+        nv = nt < ntiles ? cat_vector(p, nt, k) : none;
+        cat_load(p, nv, j, n0, n1);
 
         // ---- elements 16j..16j+15 as 8 pairs (2i, 2i+1) of this segment
         f2 y[8];
@@ -214,16 +253,15 @@ __global__ void __launch_bounds__(CAT_THREADS, 3) cat_rotate_fp8_kernel(CatRotat
 #pragma unroll
         for (int s = 0; s < 8; ++s) cb[8 * s + j] = (uint16_t)q[s];
         __syncwarp();
-        if (v >= 0) {
+        if (cv.t >= 0) {
+            const int64_t v = (int64_t)cv.t * p.G + cv.g;
             const uint4 out = *reinterpret_cast<const uint4*>(&sh.codes[k][4 * j]);
             *reinterpret_cast<uint4*>(p.out + v * 128 + 16 * j) = out;
             if (j == 0) {
-                if (p.scale_layout == 0) {
+                if (p.scale_layout == 0)
                     p.scales[v] = sc;
-                } else {
-                    const int64_t t = v / p.G;
-                    p.scales[(v - t * p.G) * p.scale_ld + t] = sc;
-                }
+                else
+                    p.scales[(int64_t)cv.g * p.scale_ld + cv.t] = sc;
             }
         }
         __syncwarp();  // the exchange buffers are reused by the next tile
@@ -322,8 +360,11 @@ __global__ void convert_kernel(int fmt, const float* in, uint8_t* out, int64_t n
 }
 
 // ------------------------------------------------------------ launchers
+int cat_rotate_group_tiles(int G) { return (G + CAT_TG - 1) / CAT_TG; }
+
 int64_t cat_rotate_tiles(const CatRotateParams& p) {
-    return p.scale_layout == 0 ? (p.nvec + CAT_VEC - 1) / CAT_VEC : p.G * ((p.M + CAT_VEC - 1) / CAT_VEC);
+    return p.scale_layout == 0 ? (p.nvec + CAT_VEC - 1) / CAT_VEC
+                               : ((p.G + CAT_TG - 1) / CAT_TG) * ((p.M + CAT_TT - 1) / CAT_TT);
 }
 
 int cat_rotate_blocks_per_sm() {

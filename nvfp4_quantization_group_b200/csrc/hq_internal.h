@@ -20,6 +20,8 @@ struct CatRotateParams {
     int64_t nvec;  // M * G vectors of 128
     int64_t M;     // rows (tokens)
     int64_t ntiles;  // tiles of 32 vectors (see cat_rotate_tiles)
+    uint32_t g_magic;      // floor((2^32 - 1) / G): v / G by multiply-high
+    uint32_t gt_magic;     // the same for the group tiles of the transposed layout
     int G;
     int rotate;    // 1: H128 / sqrt(128); 0: none
     uint8_t* out;
@@ -41,6 +43,7 @@ constexpr int K128_UNROLL = 4;      // warp steps with loads in flight
 
 int cat_rotate_blocks_per_sm();
 int64_t cat_rotate_tiles(const CatRotateParams& p);
+int cat_rotate_group_tiles(int G);  // group tiles of the transposed-scale layout
 void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st);
 void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st);
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st);
