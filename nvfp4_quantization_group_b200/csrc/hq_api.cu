@@ -276,6 +276,8 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     p.scales = scales;
     p.scale_layout = scale_layout;
     p.scale_ld = scale_ld;
+    p.wide = a_width % 16 == 0 && b_width % 16 == 0 && a_row_stride % 16 == 0 && b_row_stride % 16 == 0 &&
+             (reinterpret_cast<uintptr_t>(a) & 31u) == 0 && (b_width == 0 || (reinterpret_cast<uintptr_t>(b) & 31u) == 0);
     p.ntiles = cat_rotate_tiles(p);
     if (p.nvec >= ((int64_t)1 << 31) || p.ntiles >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
     p.g_magic = 0xFFFFFFFFu / (uint32_t)G;

@@ -131,6 +131,12 @@ __device__ __forceinline__ void cat_load(const CatRotateParams& p, CatVec cv, in
     const int64_t t = cv.t;
     const int g = cv.g;
     const int a_chunks = p.a_width / 8;
+    if (p.wide) {
+        const uint16_t* src = 2 * j < a_chunks ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + j * 16
+                                               : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (2 * j - a_chunks) * 8;
+        ld_nc_v8(src, c0, c1);
+        return;
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int c = 2 * j + h;

@@ -22,6 +22,7 @@ struct CatRotateParams {
     int64_t ntiles;  // tiles of 32 vectors (see cat_rotate_tiles)
     uint32_t g_magic;      // floor((2^32 - 1) / G): v / G by multiply-high
     uint32_t gt_magic;     // the same for the group tiles of the transposed layout
+    int wide;              // 16-element segments never straddle a and b, 32-byte aligned: 32-byte loads
     int G;
     int rotate;    // 1: H128 / sqrt(128); 0: none
     uint8_t* out;
