@@ -305,6 +305,8 @@ hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out,
     p.in = in;
     p.K_out = K_out;
     p.ngroups = M * (K_out / 128);
+    if (p.ngroups >= ((int64_t)1 << 31) || K_out / 128 >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
+    p.gpr_magic = 0xFFFFFFFFu / (uint32_t)(K_out / 128);
     p.out = out_fp8;
     p.scales = scales;
     constexpr int warps_per_block = K128_THREADS / 32;

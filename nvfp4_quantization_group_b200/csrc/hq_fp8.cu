@@ -276,43 +276,116 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_fp8_kerne
 
 // ------------------------------------------------------------ K128 quant
 // A half-warp (16 lanes x 8 values) owns one group of 128; a warp works on
-// two consecutive groups (adjacent in memory) per step and keeps UNROLL
-// steps of loads in flight before computing.
+// two consecutive groups (adjacent in memory) per step.  BF16 / FP32 input:
+// the raw load words of the next batch of steps are fetched before the
+// current batch is computed (two register buffers), so loads stay in flight
+// during the arithmetic.  SwiGLU input: compute-heavy, loads of a batch
+// first and then its arithmetic.
+template <int MODE> struct K128Raw;
+template <> struct K128Raw<HQ_ACT_NONE_BF16> { static constexpr int U = 4; uint4 w[U]; };
+template <> struct K128Raw<HQ_ACT_NONE_F32> { static constexpr int U = 2; uint4 w[U][2]; };
+
+// Scale, codes and the stores of one group whose negated values are ny.
+__device__ __forceinline__ void k128_finish(const K128Params& p, uint32_t g, bool valid, int l, const f2 (&ny)[4],
+                                            bool split_store) {
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a, b;
+        unpack2(ny[j], a, b);
+        m = absmax3(m, a, b);
+    }
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float s = fp8_group_scale(m);
+    if (valid) {
+        const uint2 c = quant8(ny, s);
+        uint8_t* out = p.out + (uint64_t)g * 128;
+        if (!split_store) {
+            *reinterpret_cast<uint2*>(out + 8 * l) = c;
+        } else {
+            *reinterpret_cast<uint32_t*>(out + 4 * l) = c.x;
+            *reinterpret_cast<uint32_t*>(out + 64 + 4 * l) = c.y;
+        }
+        if (l == 0) p.scales[g] = s;
+    }
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4, l = lane & 15;
-    const int64_t warp = ((int64_t)blockIdx.x * K128_THREADS + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * K128_THREADS) >> 5;
-    const int64_t npairs = (p.ngroups + 1) >> 1;
-    const int64_t gpr = p.K_out / 128;  // groups per row
+    const uint32_t warp = (blockIdx.x * K128_THREADS + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * K128_THREADS) >> 5;
+    const uint32_t ngroups = (uint32_t)p.ngroups;  // < 2^31 (host check)
+    const uint32_t npairs = (ngroups + 1) >> 1;
 
-    for (int64_t base = warp * K128_UNROLL; base < npairs; base += nwarps * K128_UNROLL) {
-        f2 ny[K128_UNROLL][4];
-        // ---- loads (all steps first)
+    if constexpr (MODE != HQ_ACT_SWIGLU_F32) {
+        using Raw = K128Raw<MODE>;
+        constexpr int U = Raw::U;
+        const uint32_t stride = nwarps * U;
+        auto load = [&](uint32_t base, Raw& r) {
 #pragma unroll
-        for (int u = 0; u < K128_UNROLL; ++u) {
-            const int64_t g = (base + u) * 2 + half;
-            if (base + u < npairs && g < p.ngroups) {
-                if (MODE == HQ_ACT_NONE_BF16) {
-                    const uint16_t* in = reinterpret_cast<const uint16_t*>(p.in) + g * 128 + 8 * l;
-                    uint4 w = ld_nc_v4(in);
-                    // negate both BF16 halves before widening: exact
-                    ny[u][0] = bf16x2_to_f2(w.x ^ 0x80008000u);
-                    ny[u][1] = bf16x2_to_f2(w.y ^ 0x80008000u);
-                    ny[u][2] = bf16x2_to_f2(w.z ^ 0x80008000u);
-                    ny[u][3] = bf16x2_to_f2(w.w ^ 0x80008000u);
-                } else if (MODE == HQ_ACT_NONE_F32) {
-                    const float* in = reinterpret_cast<const float*>(p.in) + g * 128;
-                    uint4 w0 = ld_nc_v4(in + 4 * l), w1 = ld_nc_v4(in + 64 + 4 * l);
-                    ny[u][0] = pack2(-__uint_as_float(w0.x), -__uint_as_float(w0.y));
-                    ny[u][1] = pack2(-__uint_as_float(w0.z), -__uint_as_float(w0.w));
-                    ny[u][2] = pack2(-__uint_as_float(w1.x), -__uint_as_float(w1.y));
-                    ny[u][3] = pack2(-__uint_as_float(w1.z), -__uint_as_float(w1.w));
+            for (int u = 0; u < U; ++u) {
+                const uint32_t g = (base + u) * 2 + half;
+                const bool ok = base + u < npairs && g < ngroups;
+                if constexpr (MODE == HQ_ACT_NONE_BF16) {
+                    r.w[u] = ok ? ld_nc_v4(reinterpret_cast<const uint16_t*>(p.in) + (uint64_t)g * 128 + 8 * l)
+                                : make_uint4(0u, 0u, 0u, 0u);
                 } else {
-                    const int64_t row = g / gpr;
-                    const int64_t col = (g - row * gpr) * 128;
-                    const float* gate = reinterpret_cast<const float*>(p.in) + row * 2 * p.K_out + col;
+                    const float* in = reinterpret_cast<const float*>(p.in) + (uint64_t)g * 128;
+                    r.w[u][0] = ok ? ld_nc_v4(in + 4 * l) : make_uint4(0u, 0u, 0u, 0u);
+                    r.w[u][1] = ok ? ld_nc_v4(in + 64 + 4 * l) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        };
+        auto compute = [&](uint32_t base, const Raw& r) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const uint32_t g = (base + u) * 2 + half;
+                const bool ok = base + u < npairs && g < ngroups;
+                f2 ny[4];
+                if constexpr (MODE == HQ_ACT_NONE_BF16) {
+                    // negate both BF16 halves before widening: exact
+                    const uint4 w = r.w[u];
+                    ny[0] = bf16x2_to_f2(w.x ^ 0x80008000u);
+                    ny[1] = bf16x2_to_f2(w.y ^ 0x80008000u);
+                    ny[2] = bf16x2_to_f2(w.z ^ 0x80008000u);
+                    ny[3] = bf16x2_to_f2(w.w ^ 0x80008000u);
+                } else {
+                    const uint4 w0 = r.w[u][0], w1 = r.w[u][1];
+                    ny[0] = pack2(-__uint_as_float(w0.x), -__uint_as_float(w0.y));
+                    ny[1] = pack2(-__uint_as_float(w0.z), -__uint_as_float(w0.w));
+                    ny[2] = pack2(-__uint_as_float(w1.x), -__uint_as_float(w1.y));
+                    ny[3] = pack2(-__uint_as_float(w1.z), -__uint_as_float(w1.w));
+                }
+                k128_finish(p, g, ok, l, ny, MODE != HQ_ACT_NONE_BF16);
+            }
+        };
+        Raw r0, r1;
+        uint32_t base = warp * U;
+        load(base, r0);
+        while (base < npairs) {
+            load(base + stride, r1);
+            compute(base, r0);
+            base += stride;
+            if (base >= npairs) break;
+            load(base + stride, r0);
+            compute(base, r1);
+            base += stride;
+        }
+    } else {
+        const uint32_t gpr = (uint32_t)(p.K_out / 128);  // groups per row
+        for (uint32_t base = warp * K128_UNROLL; base < npairs; base += nwarps * K128_UNROLL) {
+            f2 ny[K128_UNROLL][4];
+            // ---- loads and activation (all steps first)
+#pragma unroll
+            for (int u = 0; u < K128_UNROLL; ++u) {
+                const uint32_t g = (base + u) * 2 + half;
+                if (base + u < npairs && g < ngroups) {
+                    uint32_t colg;
+                    const uint32_t row = udivmod(g, gpr, p.gpr_magic, colg);
+                    const float* gate = reinterpret_cast<const float*>(p.in) + (uint64_t)row * 2 * p.K_out + colg * 128;
                     const float* up = gate + p.K_out;
                     uint4 g0 = ld_nc_v4(gate + 4 * l), g1 = ld_nc_v4(gate + 64 + 4 * l);
                     uint4 u0 = ld_nc_v4(up + 4 * l), u1 = ld_nc_v4(up + 64 + 4 * l);
@@ -324,35 +397,15 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
                         act[j] = neg_swiglu(__uint_as_float(gg[j]), __uint_as_float(uu[j]));
 #pragma unroll
                     for (int j = 0; j < 4; ++j) ny[u][j] = pack2(act[2 * j], act[2 * j + 1]);
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) ny[u][j] = 0;
-            }
-        }
-        // ---- per group: amax over 16 lanes, scale, codes
-#pragma unroll
-        for (int u = 0; u < K128_UNROLL; ++u) {
-            const int64_t g = (base + u) * 2 + half;
-            float m = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float a, b;
-                unpack2(ny[u][j], a, b);
-                m = absmax3(m, a, b);
-            }
-#pragma unroll
-            for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            const float s = fp8_group_scale(m);
-            if (base + u < npairs && g < p.ngroups) {
-                uint2 c = quant8(ny[u], s);
-                if (MODE == HQ_ACT_NONE_BF16) {
-                    *reinterpret_cast<uint2*>(p.out + g * 128 + 8 * l) = c;
                 } else {
-                    *reinterpret_cast<uint32_t*>(p.out + g * 128 + 4 * l) = c.x;
-                    *reinterpret_cast<uint32_t*>(p.out + g * 128 + 64 + 4 * l) = c.y;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) ny[u][j] = 0;
                 }
-                if (l == 0) p.scales[g] = s;
+            }
+#pragma unroll
+            for (int u = 0; u < K128_UNROLL; ++u) {
+                const uint32_t g = (base + u) * 2 + half;
+                k128_finish(p, g, base + u < npairs && g < ngroups, l, ny[u], true);
             }
         }
     }

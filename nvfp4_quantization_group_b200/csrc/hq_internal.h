@@ -34,7 +34,8 @@ struct CatRotateParams {
 struct K128Params {
     const void* in;
     int64_t K_out;
-    int64_t ngroups;  // M * K_out / 128
+    int64_t ngroups;    // M * K_out / 128 (< 2^31)
+    uint32_t gpr_magic;  // floor((2^32 - 1) / (K_out / 128)): row of a group by multiply-high
     uint8_t* out;
     float* scales;
 };
