@@ -56,17 +56,14 @@ void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid,
 // two exact power-of-two steps.  x > 88.8 -> +inf, x < -104 -> +0.
 __device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
-__device__ __forceinline__ float hq_exp(float x) {
-    if (isnan(x)) return x;
-    if (x > 88.8f) return __uint_as_float(0x7F800000u);
-    if (x < -104.0f) return 0.0f;
+__device__ __forceinline__ float hq_exp_core(float x, float& p) {
     const float LOG2E = __uint_as_float(0x3FB8AA3Bu);
     const float LN2_HI = __uint_as_float(0x3F317200u);
     const float LN2_LO = __uint_as_float(0x35BFBE8Eu);
     const float k = rintf(__fmul_rn(x, LOG2E));
     float r = __fmaf_rn(-k, LN2_HI, x);
     r = __fmaf_rn(-k, LN2_LO, r);
-    float p = __uint_as_float(0x39500D01u);            // RN(1/5040)
+    p = __uint_as_float(0x39500D01u);                  // RN(1/5040)
     p = __fmaf_rn(p, r, __uint_as_float(0x3AB60B61u)); // RN(1/720)
     p = __fmaf_rn(p, r, __uint_as_float(0x3C088889u)); // RN(1/120)
     p = __fmaf_rn(p, r, __uint_as_float(0x3D2AAAABu)); // RN(1/24)
@@ -74,7 +71,22 @@ __device__ __forceinline__ float hq_exp(float x) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    const int ki = (int)k;
+    return k;
+}
+
+__device__ __forceinline__ float hq_exp(float x) {
+    // |x| < 87 (NaN fails the test): k = rint(x log2 e) lies in [-126, 126]
+    // and the scaling is one exact step, the same operations as below
+    if (fabsf(x) < 87.0f) {
+        float p;
+        const float k = hq_exp_core(x, p);
+        return __fmul_rn(p, pow2i((int)k));
+    }
+    if (isnan(x)) return x;
+    if (x > 88.8f) return __uint_as_float(0x7F800000u);
+    if (x < -104.0f) return 0.0f;
+    float p;
+    const int ki = (int)hq_exp_core(x, p);
     if (ki > 127) return __fmul_rn(__fmul_rn(p, pow2i(127)), pow2i(ki - 127));
     if (ki < -126) return __fmul_rn(__fmul_rn(p, pow2i(ki + 100)), pow2i(-100));
     return __fmul_rn(p, pow2i(ki));
