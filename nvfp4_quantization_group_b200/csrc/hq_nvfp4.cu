@@ -73,6 +73,8 @@ struct alignas(16) StageHdr {  // 48 bytes, moved as three 16-byte words
 
 struct NvShared {
     float2 vr[128];  // per E4M3 code: {value, -RN(1 / value)}; {0, -0} for codes 0 and 127
+    float enc[NST][2][128];  // per buffer: S_enc / value(sf) for every code, rowwise and columnwise
+    int32_t enc_section[NST];  // section the buffer's tables hold (producer only)
     StageHdr hdr[NST];
     uint32_t acc_row[NST], acc_col[NST], acc_cnt[NST];  // amax tiles: CTA partial maxima
     uint32_t seg_start[NV_MAX_SEG + 1];  // copies of the schedule (parameter space is slow
@@ -353,6 +355,17 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
         if (lane == 0) claim = atomicAdd(counter, 1u);
         const TileInfo t = k == 1u ? decode(p, sh, tile, ps.seg) : ps.nt;
         const uint32_t fl = nv_prepare(p, h, t, lane, ps);
+        if ((fl & H_CAST) && !(fl & H_GAVE_UP) && sh.enc_section[st] != t.s) {
+            // this buffer's encode tables for the section (each lane writes and
+            // later reads only the value it wrote itself into enc_section)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t code = (uint32_t)lane + 32u * m;
+                sh.enc[st][0][code] = block_enc(sh, code, ps.r_sr, fl & H_SLOW_R);
+                sh.enc[st][1][code] = block_enc(sh, code, ps.r_scq, fl & H_SLOW_C);
+            }
+            sh.enc_section[st] = t.s;
+        }
         if (lane == 0 && !(fl & H_GAVE_UP)) {
             const uint32_t dst = tiles_u32 + (uint32_t)st * TILE_BYTES;
             const int c1 = (int)(t.row0 / 16);
@@ -506,7 +519,6 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             for (int vw = w; vw < 16; vw += NCW) {
             const Part pt = part(vw);
             if (do_row) {
-                const bool slow = h.flags & H_SLOW_R;
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const uint32_t ro = pt.roff0 + 4096u * kk;
@@ -516,7 +528,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     const uint32_t m = hmax_abs(hmax_abs(hmax_abs(wd[0], wd[1]), hmax_abs(wd[2], wd[3])),
                                                 hmax_abs(hmax_abs(wd[4], wd[5]), hmax_abs(wd[6], wd[7])));
                     const uint32_t sf = block_sf(__uint_as_float(halves_max_bits(m)), h.senc_r);
-                    const float enc = block_enc(sh, sf, h.senc_r, slow);
+                    const float enc = sh.enc[st][0][sf];
                     const f2 e2 = pack2(enc, enc);
                     float q[16];
 #pragma unroll
@@ -550,8 +562,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 }
                 const uint32_t sf0 = block_sf(__fmul_rn(a0, 0.25f), h.senc_c);
                 const uint32_t sf1 = block_sf(__fmul_rn(a1, 0.25f), h.senc_c);
-                const bool slow = h.flags & H_SLOW_C;
-                const f2 e2 = pack2(block_enc(sh, sf0, h.senc_cq, slow), block_enc(sh, sf1, h.senc_cq, slow));
+                const f2 e2 = pack2(sh.enc[st][1][sf0], sh.enc[st][1][sf1]);
                 if (!(h.flags & H_FOLD)) {
                     const f2 quarter = pack2(0.25f, 0.25f);
 #pragma unroll
@@ -604,6 +615,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
             sh.acc_row[st] = 0u;
             sh.acc_col[st] = 0u;
             sh.acc_cnt[st] = 0u;
+            sh.enc_section[st] = -1;
         }
         fence_mbar_init();
     }
