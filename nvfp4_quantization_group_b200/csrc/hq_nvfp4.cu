@@ -146,6 +146,20 @@ __device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t
     }
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// max |x| over 16 values, as a tree of depth 3 (max is exact: any order gives
+// the same value)
+__device__ __forceinline__ float absmax16(const float (&x)[16]) {
+    const float a = max3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2])), b = max3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+    const float c = max3(fabsf(x[6]), fabsf(x[7]), fabsf(x[8])), d = max3(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
+    const float e = max3(fabsf(x[12]), fabsf(x[13]), fabsf(x[14]));
+    return max3(max3(a, b, c), max3(d, e, fabsf(x[15])), 0.0f);
+}
+
 // Shared byte offset of 16-byte chunk q (0..7) of column half h of tile row
 // 16 rb + i.
 __device__ __forceinline__ uint32_t chunk_off(int h, int rb, int i, int q) {
@@ -474,12 +488,10 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + pt.coff + 1024 * i);
                 f2 v[16];
                 column_rht(x, sg, v);
+                float c0[16], c1[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float a0, a1;
-                    unpack2(v[i], a0, a1);
-                    mcol = absmax3(mcol, a0, a1);
-                }
+                for (int i = 0; i < 16; ++i) unpack2(v[i], c0[i], c1[i]);
+                mcol = max3(mcol, absmax16(c0), absmax16(c1));
             }
             }  // parts
 #pragma unroll
@@ -551,15 +563,10 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + pt.coff + 1024 * i);
                 f2 v[16];
                 column_rht(x, sg, v);
-                float a0 = 0.0f, a1 = 0.0f;
+                float c0[16], c1[16];
 #pragma unroll
-                for (int i = 0; i < 16; i += 2) {
-                    float x0, x1, y0, y1;
-                    unpack2(v[i], x0, x1);
-                    unpack2(v[i + 1], y0, y1);
-                    a0 = absmax3(a0, x0, y0);
-                    a1 = absmax3(a1, x1, y1);
-                }
+                for (int i = 0; i < 16; ++i) unpack2(v[i], c0[i], c1[i]);
+                const float a0 = absmax16(c0), a1 = absmax16(c1);
                 const uint32_t sf0 = block_sf(__fmul_rn(a0, 0.25f), h.senc_c);
                 const uint32_t sf1 = block_sf(__fmul_rn(a1, 0.25f), h.senc_c);
                 const f2 e2 = pack2(sh.enc[st][1][sf0], sh.enc[st][1][sf1]);
