@@ -469,7 +469,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             // ===================================================== amax tile
             uint32_t mrow = 0u;
             float mcol = 0.0f;
-            for (int vw = w; vw < 16; vw += NCW) {
+#pragma unroll
+            for (int pi = 0; pi < 16 / NCW; ++pi) {
+            const int vw = w + pi * NCW;
             const Part pt = part(vw);
             if (do_row) {
 #pragma unroll
@@ -528,7 +530,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             // ===================================================== cast tile
             uint8_t* const rc_base = p.row_codes + (uint64_t)h.row0 * K2 + (uint32_t)h.col0 / 2u;
             uint8_t* const rs_base = p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
-            for (int vw = w; vw < 16; vw += NCW) {
+#pragma unroll
+            for (int pi = 0; pi < 16 / NCW; ++pi) {
+            const int vw = w + pi * NCW;
             const Part pt = part(vw);
             if (do_row) {
 #pragma unroll
