@@ -76,11 +76,27 @@ __device__ __forceinline__ float hq_exp_core(float x, float& p) {
 
 __device__ __forceinline__ float hq_exp(float x) {
     // |x| < 87 (NaN fails the test): k = rint(x log2 e) lies in [-126, 126]
-    // and the scaling is one exact step, the same operations as below
+    // and the scaling is one exact step, the same operations as below.  Here
+    // rint is the addition of 1.5 * 2^23 (round to nearest even, exact for
+    // |t| < 2^22), whose bits also give k and 2^k as integers.
     if (fabsf(x) < 87.0f) {
-        float p;
-        const float k = hq_exp_core(x, p);
-        return __fmul_rn(p, pow2i((int)k));
+        const float LOG2E = __uint_as_float(0x3FB8AA3Bu);
+        const float LN2_HI = __uint_as_float(0x3F317200u);
+        const float LN2_LO = __uint_as_float(0x35BFBE8Eu);
+        const float big = __fadd_rn(__fmul_rn(x, LOG2E), 12582912.0f);  // 1.5 * 2^23 + rint(x log2 e)
+        const float k = __fsub_rn(big, 12582912.0f);
+        float r = __fmaf_rn(-k, LN2_HI, x);
+        r = __fmaf_rn(-k, LN2_LO, r);
+        float p = __uint_as_float(0x39500D01u);                  // RN(1/5040)
+        p = __fmaf_rn(p, r, __uint_as_float(0x3AB60B61u)); // RN(1/720)
+        p = __fmaf_rn(p, r, __uint_as_float(0x3C088889u)); // RN(1/120)
+        p = __fmaf_rn(p, r, __uint_as_float(0x3D2AAAABu)); // RN(1/24)
+        p = __fmaf_rn(p, r, __uint_as_float(0x3E2AAAABu)); // RN(1/6)
+        p = __fmaf_rn(p, r, 0.5f);
+        p = __fmaf_rn(p, r, 1.0f);
+        p = __fmaf_rn(p, r, 1.0f);
+        const uint32_t two_k = (__float_as_uint(big) - 0x4B400000u + 127u) << 23;  // bits of 2^k
+        return __fmul_rn(p, __uint_as_float(two_k));
     }
     if (isnan(x)) return x;
     if (x > 88.8f) return __uint_as_float(0x7F800000u);
