@@ -167,11 +167,14 @@ def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False):
     return out, scales, pre
 
 
-ROWWISE, COLWISE = 1, 2
+ROWWISE, COLWISE, ROW_RHT = 1, 2, 4
 
 
 def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=False):
     """Grouped RHT16 + NVFP4 cast.  x: uint16 BF16 bits [M, K].
+
+    ROW_RHT (with ROWWISE) rotates every 16-element row block along K before
+    the rowwise amax and cast.
 
     Returns a dict with row_codes [M, K/2], row_sf [M, K/16], col_codes
     [M*K/2], col_sf [M*K/16] (sections concatenated, each [K, M_s/...]),

@@ -419,6 +419,11 @@ static void rht16(const float *x, uint16_t sign_mask, float *v)
  * [FUS]'s fusion rule; K a multiple of 128).
  * flags bit 0 (rowwise): plain cast of x along K (the pages' rowwise output
  *   carries no RHT):  row_codes [M, K/2], row_sf [M, K/16].
+ * flags bit 2 (with bit 0): the rowwise output instead casts the 16-point RHT
+ *   of every 16-element row block along K (the same sign mask, sigma by the
+ *   position inside the block): the other reading of "RHT ... rowwise and
+ *   columnwise"; section amax and block scales then come from the rotated
+ *   values.
  * flags bit 1 (columnwise): per section, the 16-point RHT along M (16
  *   consecutive rows of one column), cast, stored transposed: section s
  *   starting at row r0 owns col_codes[K*r0/2 ...] as [K, M_s/2] and
@@ -449,18 +454,29 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
     for (int s = 0; s < S; ++s) {
         const int64_t Ms = split_rows[s];
         if (flags & 1) {
+            const int rotate = (flags & 4) != 0;
+            /* first pass: section amax (of the rotated blocks if rotating) */
             float A = 0.0f;
-            for (int64_t r = r0; r < r0 + Ms; ++r)
-                for (int64_t k = 0; k < K; ++k)
-                    A = fmaxf(A, fabsf(bf16_value(x[r * K + k])));
-            float S_enc = global_encode_scale(A);
-            amax_row[s] = A;
-            sdec_row[s] = 1.0f / S_enc;
             for (int64_t r = r0; r < r0 + Ms; ++r)
                 for (int64_t kb = 0; kb < K / 16; ++kb) {
                     for (int i = 0; i < 16; ++i)
                         blk[i] = bf16_value(x[r * K + kb * 16 + i]);
-                    nvfp4_block(blk, S_enc, row_codes + r * (K / 2) + kb * 8,
+                    if (rotate)
+                        rht16(blk, sign_mask, v);
+                    for (int i = 0; i < 16; ++i)
+                        A = fmaxf(A, fabsf(rotate ? v[i] : blk[i]));
+                }
+            float S_enc = global_encode_scale(A);
+            amax_row[s] = A;
+            sdec_row[s] = 1.0f / S_enc;
+            /* second pass: cast */
+            for (int64_t r = r0; r < r0 + Ms; ++r)
+                for (int64_t kb = 0; kb < K / 16; ++kb) {
+                    for (int i = 0; i < 16; ++i)
+                        blk[i] = bf16_value(x[r * K + kb * 16 + i]);
+                    if (rotate)
+                        rht16(blk, sign_mask, v);
+                    nvfp4_block(rotate ? v : blk, S_enc, row_codes + r * (K / 2) + kb * 8,
                                 row_sf + r * (K / 16) + kb,
                                 row_pre ? row_pre + r * K + kb * 16 : 0);
                 }

@@ -441,6 +441,62 @@ def test_nvfp4_flags_select_directions_and_reject_bad_splits():
         oracle.group_rht_quant(x, [128], 0, oracle.ROWWISE)           # splits do not sum to M
 
 
+def test_nvfp4_row_rht_is_rotation_along_k():
+    """ROW_RHT: every 16-element row block is rotated (sigma by position in the
+    block) before the rowwise amax and cast; checked against a dense FP64
+    rotation, the inverse rotation of the dequantized rows and the plain cast
+    when the flag is off."""
+    x, splits, mask = _nvfp4_case(seed=83, splits=(256, 128, 0))
+    r = oracle.group_rht_quant(x, splits, mask, oracle.ROWWISE | oracle.ROW_RHT, want_pre=True)
+    plain = oracle.group_rht_quant(x, splits, mask, oracle.ROWWISE)
+    assert not np.array_equal(r["row_codes"], plain["row_codes"])
+    xf = S.bf16_bits_to_f32(x).astype(np.float64)
+    M, K = x.shape
+    H = scipy.linalg.hadamard(16).astype(np.float64)
+    sigma = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+    r0 = 0
+    for s, Ms in enumerate(splits):
+        if Ms == 0:
+            assert r["amax_row"][s] == 0 and r["sdec_row"][s] == 1
+            continue
+        blocks = xf[r0:r0 + Ms].reshape(Ms, K // 16, 16)
+        v_ref = _rht_dense(blocks, mask)
+        A = r["amax_row"][s]
+        assert abs(A - np.max(np.abs(v_ref))) <= 1e-6 * A
+        S_enc = np.float32(2688) / A
+        assert r["sdec_row"][s] == np.float32(1) / S_enc
+        sf = r["row_sf"][r0:r0 + Ms]
+        sff = _e4m3_vals(sf)
+        enc = np.where(sff == 0, 0, np.float64(S_enc) / sff)
+        pre = r["row_pre"][r0:r0 + Ms].reshape(Ms, K // 16, 16)
+        v = pre / np.where(enc == 0, 1, enc)[..., None]
+        norms = np.linalg.norm(blocks, axis=-1, keepdims=True)
+        assert np.max(np.abs(v - v_ref) / np.maximum(norms, 1e-30)) <= 1e-5
+        # block scales follow the rotated block maxima
+        ab = np.max(np.abs(v_ref), axis=-1)
+        i, kb = np.unravel_index(np.argmax(ab), ab.shape)
+        assert sf[i, kb] == 0x7E
+        nib = _unpack(r["row_codes"][r0:r0 + Ms]).reshape(Ms, K // 16, 16)
+        deq = _e2m1_vals(nib) * sff[..., None] / np.float64(S_enc)
+        back = (0.25 * deq @ H) * sigma
+        err = np.linalg.norm(back - blocks, axis=-1)
+        assert np.all(err <= 4 * ab / 6 * 1.07 + 1e-30)
+        r0 += Ms
+
+
+def test_nvfp4_row_rht_equals_column_rht_of_transpose():
+    """Rotating rows along K of x is the columnwise transform of x^T (one
+    section each way), whose transposed output is laid out like x's rows."""
+    x = S.normal_bf16(85, (128, 256))
+    mask = 0x5A3C
+    r = oracle.group_rht_quant(x, [128], mask, oracle.ROWWISE | oracle.ROW_RHT)
+    xt = np.ascontiguousarray(x.T)
+    c = oracle.group_rht_quant(xt, [256], mask, oracle.COLWISE)
+    np.testing.assert_array_equal(r["row_codes"].reshape(-1), c["col_codes"])
+    np.testing.assert_array_equal(r["row_sf"].reshape(-1), c["col_sf"])
+    assert r["amax_row"][0] == c["amax_col"][0] and r["sdec_row"][0] == c["sdec_col"][0]
+
+
 def test_nvfp4_zero_section_and_tiny_values():
     x = np.zeros((256, 128), dtype=np.uint16)
     x[128:] = S.normal_bf16(97, (128, 128))
