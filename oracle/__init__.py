@@ -60,9 +60,9 @@ def lib() -> ctypes.CDLL:
             L.hqo_fwht.argtypes = [P, ctypes.c_int]
             L.hqo_fwht.restype = None
             L.hqo_cat_rotate_fp8.argtypes = [P, i64, ctypes.c_int, P, i64, ctypes.c_int, i64,
-                                             ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, i64, P]
+                                             ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, i64, P, P]
             L.hqo_cat_rotate_fp8.restype = ctypes.c_int
-            L.hqo_swiglu_fp8_k128.argtypes = [ctypes.c_int, P, i64, i64, P, P, P]
+            L.hqo_swiglu_fp8_k128.argtypes = [ctypes.c_int, P, i64, i64, P, P, P, P]
             L.hqo_swiglu_fp8_k128.restype = ctypes.c_int
             L.hqo_group_rht_quant.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_uint16, ctypes.c_uint,
                                               P, P, P, P, P, P, P, P, P, P]
@@ -122,11 +122,12 @@ ROWMAJOR, TRANSPOSED = 0, 1
 
 
 def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=None,
-                   scale_layout=ROWMAJOR, scale_ld=None, want_pre=False):
+                   scale_layout=ROWMAJOR, scale_ld=None, want_pre=False, want_amax=False):
     """Concat (a | b) per group, optional 128-point Hadamard, FP8 1x128 quant.
 
     a, b: uint16 BF16 bit arrays; a_width = a.shape[-1] (b may be None).
-    Returns (codes [M, G*128] uint8, scales, pre or None).
+    Returns (codes [M, G*128] uint8, scales, pre or None), and with want_amax
+    a fourth item: the groups' amax in the scales' layout.
     """
     a = np.ascontiguousarray(a, dtype=np.uint16)
     a_w = int(a.shape[-1])
@@ -145,26 +146,31 @@ def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=N
         ld = scale_ld if scale_ld is not None else M
         scales = np.zeros((G, ld), dtype=np.float32)
     pre = np.empty((M, G * 128), dtype=np.float32) if want_pre else None
+    amax = np.zeros_like(scales) if want_amax else None
     rc = lib().hqo_cat_rotate_fp8(_ptr(a), a_rs, a_w, _ptr(b), b_rs, b_w, M, G, hadamard_n,
-                                  _ptr(out), _ptr(scales), scale_layout, ld, _ptr(pre))
+                                  _ptr(out), _ptr(scales), scale_layout, ld, _ptr(amax), _ptr(pre))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
-    return out, scales, pre
+    return (out, scales, pre, amax) if want_amax else (out, scales, pre)
 
 
 NONE_BF16, NONE_F32, SWIGLU_F32 = 0, 1, 2
 
 
-def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False):
-    """K128 FP8 quantization of BF16/FP32 rows or of SiLU(gate) * up."""
+def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False, want_amax=False):
+    """K128 FP8 quantization of BF16/FP32 rows or of SiLU(gate) * up.
+
+    Returns (codes, scales, pre or None), and with want_amax a fourth item:
+    the groups' amax [M, K_out/128]."""
     x = np.ascontiguousarray(x)
     out = np.empty((M, K_out), dtype=np.uint8)
     scales = np.empty((M, K_out // 128), dtype=np.float32)
     pre = np.empty((M, K_out), dtype=np.float32) if want_pre else None
-    rc = lib().hqo_swiglu_fp8_k128(mode, _ptr(x), M, K_out, _ptr(out), _ptr(scales), _ptr(pre))
+    amax = np.empty_like(scales) if want_amax else None
+    rc = lib().hqo_swiglu_fp8_k128(mode, _ptr(x), M, K_out, _ptr(out), _ptr(scales), _ptr(amax), _ptr(pre))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
-    return out, scales, pre
+    return (out, scales, pre, amax) if want_amax else (out, scales, pre)
 
 
 ROWWISE, COLWISE, ROW_RHT = 1, 2, 4

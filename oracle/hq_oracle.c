@@ -187,9 +187,9 @@ static float c128(void)
  * The page says "FP32 div.full normalization" and notes that the choice of
  * division changes codes by one ulp at FP8 midpoints.  Reading: correctly
  * rounded IEEE division.  `pre`, when given, receives y_i / s (the value that
- * is rounded to E4M3).
+ * is rounded to E4M3); `amax_out`, when given, receives amax.
  */
-static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, float *pre)
+static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, float *amax_out, float *pre)
 {
     float amax = 0.0f;
     for (int i = 0; i < n; ++i)
@@ -203,6 +203,8 @@ static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, flo
         q[i] = hqo_e4m3_encode(t);
     }
     *scale = s;
+    if (amax_out)
+        *amax_out = amax;
 }
 
 /*
@@ -213,14 +215,15 @@ static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, flo
  * Element (t, g, j) of a is a[t * a_row_stride + g * a_width + j]; b likewise.
  * Output codes: out[(t * G + g) * 128 + j].  Scales: scale_layout 0 (row
  * major) puts group (t, g) at scales[t * G + g]; layout 1 (transposed, as the
- * indexer stores them) at scales[g * scale_ld + t].
+ * indexer stores them) at scales[g * scale_ld + t].  amax_opt, when given,
+ * receives each group's amax in the scales' layout.
  * Returns 0, or -1 for arguments this reference does not accept.
  */
 int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
                        const uint16_t *b, int64_t b_row_stride, int b_width,
                        int64_t M, int G, int hadamard_n,
                        uint8_t *out, float *scales, int scale_layout, int64_t scale_ld,
-                       float *pre)
+                       float *amax_opt, float *pre)
 {
     if (a_width < 0 || b_width < 0 || a_width + b_width != 128 || (b_width > 0 && !b))
         return -1;
@@ -240,12 +243,12 @@ int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
                     v[j] = v[j] * c;
             }
             int64_t grp = t * G + g;
-            float s;
-            quant_group_fp8(v, 128, out + grp * 128, &s, pre ? pre + grp * 128 : 0);
-            if (scale_layout == 0)
-                scales[grp] = s;
-            else
-                scales[(int64_t)g * scale_ld + t] = s;
+            float s, am;
+            quant_group_fp8(v, 128, out + grp * 128, &s, &am, pre ? pre + grp * 128 : 0);
+            const int64_t si = scale_layout == 0 ? grp : (int64_t)g * scale_ld + t;
+            scales[si] = s;
+            if (amax_opt)
+                amax_opt[si] = am;
         }
     return 0;
 }
@@ -326,10 +329,11 @@ static float swiglu(float g, float u)
  *   mode 2: in is FP32 [M, 2*K_out]; gate = columns 0..K_out-1, up = columns
  *           K_out..2*K_out-1 ("2x2048": the reading is two halves, not an
  *           interleave); the quantized value is SiLU(gate) * up.
- * out: [M, K_out] codes; scales: [M, K_out/128] row major.
+ * out: [M, K_out] codes; scales (and amax_opt, when given, each group's
+ * amax): [M, K_out/128] row major.
  */
 int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
-                        uint8_t *out, float *scales, float *pre)
+                        uint8_t *out, float *scales, float *amax_opt, float *pre)
 {
     if (K_out % 128 != 0 || mode < 0 || mode > 2)
         return -1;
@@ -349,7 +353,8 @@ int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
                 }
             }
             int64_t grp = m * groups + g;
-            quant_group_fp8(y, 128, out + grp * 128, &scales[grp], pre ? pre + grp * 128 : 0);
+            quant_group_fp8(y, 128, out + grp * 128, &scales[grp], amax_opt ? &amax_opt[grp] : 0,
+                            pre ? pre + grp * 128 : 0);
         }
     return 0;
 }

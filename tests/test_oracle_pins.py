@@ -265,6 +265,35 @@ def test_exp_within_two_ulp_of_fp64():
     assert np.isnan(oracle.exp_f32(np.float32([np.nan]))[0])
 
 
+def test_fp8_amax_outputs():
+    """amax_opt: max |y| of each group (exact max |x| without rotation; the
+    dense FP64 rotation's maximum within FP32 rounding with it), stored in the
+    scales' layout, with s = max(amax, 1e-10) * RN(1/448) in binary32."""
+    M, G = 12, 3
+    xa = S.normal_bf16(301, (M, G, 64))
+    xb = S.normal_bf16(302, (M, G, 64))
+    xa[5, 1] = 0
+    xb[5, 1] = 0                                   # an all-zero group
+    inv = np.float32(1) / np.float32(448)
+    _, sc, _, am = oracle.cat_rotate_fp8(xa, xb, M, G, 0, want_amax=True)
+    v = np.concatenate([S.bf16_bits_to_f32(xa), S.bf16_bits_to_f32(xb)], axis=-1)
+    np.testing.assert_array_equal(am, np.max(np.abs(v), axis=-1))
+    np.testing.assert_array_equal(sc, np.maximum(am, np.float32(1e-10)) * inv)
+    assert am[5, 1] == 0
+    _, sct, _, amt = oracle.cat_rotate_fp8(xa, xb, M, G, 128, scale_layout=oracle.TRANSPOSED,
+                                           scale_ld=16, want_amax=True)
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128)
+    ref = np.max(np.abs(v.astype(np.float64) @ H.T), axis=-1)      # [M, G]
+    assert amt.shape == (G, 16)
+    np.testing.assert_allclose(amt[:, :M].T, ref, rtol=2e-6)
+    assert np.all(amt[:, M:] == 0)
+    np.testing.assert_array_equal(sct[:, :M], np.maximum(amt[:, :M], np.float32(1e-10)) * inv)
+    x = S.normal_f32(303, (4, 512))
+    _, s1, _, a1 = oracle.swiglu_fp8_k128(oracle.NONE_F32, x, 4, 512, want_amax=True)
+    np.testing.assert_array_equal(a1, np.max(np.abs(x.reshape(4, 4, 128)), axis=-1))
+    np.testing.assert_array_equal(s1, np.maximum(a1, np.float32(1e-10)) * inv)
+
+
 def test_swiglu_k128_values_and_rule():
     M, K = 6, 256
     gu = S.normal_f32(51, (M, 2 * K), std=math.sqrt(2.0))
