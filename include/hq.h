@@ -56,6 +56,8 @@ typedef enum hq_status {
 /* hq_group_rht_quant flags */
 #define HQ_ROWWISE 1u      /* rowwise NVFP4 output (plain cast along K) */
 #define HQ_COLWISE 2u      /* columnwise NVFP4 output (RHT16 along M, transposed) */
+#define HQ_ROW_RHT 4u      /* with HQ_ROWWISE: the rowwise output casts the RHT16
+                              of each 16-column block along K instead of x */
 #define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
                               instead of one launch in which each section's
                               cast follows its amax while the rows are still
@@ -120,12 +122,16 @@ hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *strea
  *             128 ([FUS] fusion rule), summing to M.  Empty sections allowed.
  *  S          number of sections, 1 <= S <= HQ_MAX_SECTIONS.
  *  sign_mask  the random sign vector of the 16-point RHT: bit i set means
- *             sigma_i = -1 for position i of each 16-row block.
- *  flags      HQ_ROWWISE | HQ_COLWISE (at least one), optionally HQ_TWO_PASS.
+ *             sigma_i = -1 for position i of each 16-row block (and, with
+ *             HQ_ROW_RHT, of each 16-column block of a row).
+ *  flags      HQ_ROWWISE | HQ_COLWISE (at least one), optionally HQ_ROW_RHT
+ *             (only with HQ_ROWWISE; the grouped-quant pages speak of the RHT
+ *             on both outputs, their fused kernel rotates only the columns)
+ *             and HQ_TWO_PASS.
  *
  * For section s (rows [r0, r0 + M_s)) and each requested direction:
- *   A_s = max |v| over the section's values (v = x rowwise; v = RHT16 output
- *   columnwise), S_enc = 2688 / A_s (1 when A_s == 0 or not finite),
+ *   A_s = max |v| over the section's values (v = x rowwise, the RHT16 output
+ *   along K with HQ_ROW_RHT; v = RHT16 output columnwise), S_enc = 2688 / A_s (1 when A_s == 0 or not finite),
  *   sdec = 1 / S_enc; for each block of 16 values along the quantized
  *   direction: sf = E4M3((a_b / 6) * S_enc), code_i = E2M1(v_i * S_enc / sf)
  *   (0 when sf == 0); saturating round-to-nearest-even conversions.
@@ -199,7 +205,10 @@ hq_status hq_group_rht_quant_noalloc(const void *x, int64_t M, int64_t K,
  *             codes = E4M3(y / s) (IEEE division, saturating RNE).
  *             scale_layout HQ_SCALE_ROWMAJOR: [M, G] (scale_ld ignored);
  *             HQ_SCALE_TRANSPOSED: [G, scale_ld], scale_ld >= M.
- *  ws, ws_bytes  unused (the call needs no workspace; may be NULL / 0).
+ *  amax_opt   float, NULL or each group's amax = max |y| (y the rotated
+ *             128-vector), in the scales' layout; 4-byte aligned.
+ *  ws, ws_bytes  unused: hq_cat_rotate_fp8_workspace_size() is 0 (may be
+ *             NULL / 0).
  * Alignment: a, b, out 16 bytes; strides multiples of 8 elements.
  * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
  *         HQ_ERR_CUDA.
@@ -208,7 +217,11 @@ hq_status hq_cat_rotate_fp8(const void *a, int64_t a_row_stride, int a_width,
                             const void *b, int64_t b_row_stride, int b_width,
                             int64_t M, int G, int hadamard_n,
                             uint8_t *out_fp8, float *scales, int scale_layout,
-                            int64_t scale_ld, void *ws, size_t ws_bytes, void *stream);
+                            int64_t scale_ld, float *amax_opt,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes hq_cat_rotate_fp8 needs: 0 (none). */
+size_t hq_cat_rotate_fp8_workspace_size(void);
 
 /*
  * QMoE dynamic FP8 activation quantizer [QMOE]: each row of K_out values is
@@ -218,14 +231,19 @@ hq_status hq_cat_rotate_fp8(const void *a, int64_t a_row_stride, int a_width,
  *           g / (1 + exp(-g)), with no narrower rounding in between).
  *  in       see the modes; row stride K_out (or 2*K_out for SwiGLU).
  *  out_fp8  uint8 [M, K_out];  scales float [M, K_out/128] row major.
- *  K_out    multiple of 128.   ws, ws_bytes unused (may be NULL / 0).
- * Alignment: in and out 16 bytes, scales 4 bytes.
+ *  amax_opt float [M, K_out/128] or NULL: each group's amax = max |y|.
+ *  K_out    multiple of 128.   ws, ws_bytes unused:
+ *           hq_swiglu_fp8_k128_workspace_size() is 0 (may be NULL / 0).
+ * Alignment: in and out 16 bytes, scales and amax_opt 4 bytes.
  * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
  *         HQ_ERR_CUDA.
  */
 hq_status hq_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
-                             uint8_t *out_fp8, float *scales,
+                             uint8_t *out_fp8, float *scales, float *amax_opt,
                              void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes hq_swiglu_fp8_k128 needs: 0 (none). */
+size_t hq_swiglu_fp8_k128_workspace_size(void);
 
 /*
  * Element-wise conversion of FP32 values with the library's own device

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libhq.so")
 
 HQ_OK, HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA, \
     HQ_ERR_TIMEOUT = range(8)
-HQ_ROWWISE, HQ_COLWISE, HQ_TWO_PASS = 1, 2, 8
+HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS = 1, 2, 4, 8
 HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
 HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
 HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1
@@ -30,8 +30,8 @@ HQ_MAX_SECTIONS = 256
 
 EXPORTED = (
     "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
-    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8", "hq_swiglu_fp8_k128",
-    "hq_convert",
+    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8",
+    "hq_cat_rotate_fp8_workspace_size", "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
 )
 
 
@@ -71,9 +71,13 @@ def lib() -> ctypes.CDLL:
                                                  P, P, P, P, P, P, P, P, P]
         L.hq_cat_rotate_fp8.restype = c_int
         L.hq_cat_rotate_fp8.argtypes = [P, i64, c_int, P, i64, c_int, i64, c_int, c_int,
-                                        P, P, c_int, i64, P, sz, P]
+                                        P, P, c_int, i64, P, P, sz, P]
+        L.hq_cat_rotate_fp8_workspace_size.restype = sz
+        L.hq_cat_rotate_fp8_workspace_size.argtypes = []
         L.hq_swiglu_fp8_k128.restype = c_int
-        L.hq_swiglu_fp8_k128.argtypes = [c_int, P, i64, i64, P, P, P, sz, P]
+        L.hq_swiglu_fp8_k128.argtypes = [c_int, P, i64, i64, P, P, P, P, sz, P]
+        L.hq_swiglu_fp8_k128_workspace_size.restype = sz
+        L.hq_swiglu_fp8_k128_workspace_size.argtypes = []
         L.hq_convert.restype = c_int
         L.hq_convert.argtypes = [c_int, P, P, i64, P]
         _lib = L
@@ -147,16 +151,24 @@ def hq_group_rht_quant_noalloc(x, M, K, split_rows, S, sign_mask, flags, row_cod
 
 
 def hq_cat_rotate_fp8(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, out_fp8, scales,
-                      scale_layout, scale_ld, stream=None) -> None:
+                      scale_layout, scale_ld, amax_opt=None, stream=None) -> None:
     _check(lib().hq_cat_rotate_fp8(_p(a), int(a_row_stride), int(a_width), _p(b), int(b_row_stride),
                                    int(b_width), int(M), int(G), int(hadamard_n), _p(out_fp8), _p(scales),
-                                   int(scale_layout), int(scale_ld), None, 0, _stream(stream)),
+                                   int(scale_layout), int(scale_ld), _p(amax_opt), None, 0, _stream(stream)),
            "hq_cat_rotate_fp8")
 
 
-def hq_swiglu_fp8_k128(mode, inp, M, K_out, out_fp8, scales, stream=None) -> None:
-    _check(lib().hq_swiglu_fp8_k128(int(mode), _p(inp), int(M), int(K_out), _p(out_fp8), _p(scales), None, 0,
-                                    _stream(stream)), "hq_swiglu_fp8_k128")
+def hq_cat_rotate_fp8_workspace_size() -> int:
+    return int(lib().hq_cat_rotate_fp8_workspace_size())
+
+
+def hq_swiglu_fp8_k128(mode, inp, M, K_out, out_fp8, scales, amax_opt=None, stream=None) -> None:
+    _check(lib().hq_swiglu_fp8_k128(int(mode), _p(inp), int(M), int(K_out), _p(out_fp8), _p(scales),
+                                    _p(amax_opt), None, 0, _stream(stream)), "hq_swiglu_fp8_k128")
+
+
+def hq_swiglu_fp8_k128_workspace_size() -> int:
+    return int(lib().hq_swiglu_fp8_k128_workspace_size())
 
 
 def hq_convert(fmt, inp, out, n, stream=None) -> None:
@@ -203,8 +215,10 @@ def group_rht_quant(x: torch.Tensor, split_rows, sign_mask: int, flags: int = HQ
 
 
 def cat_rotate_fp8(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 128,
-                   scale_layout: int = HQ_SCALE_ROWMAJOR, scale_ld: int | None = None, stream=None):
-    """a: BF16 [M, G, a_width], b: BF16 [M, G, b_width] or None -> (codes [M, G*128], scales)."""
+                   scale_layout: int = HQ_SCALE_ROWMAJOR, scale_ld: int | None = None, want_amax: bool = False,
+                   stream=None):
+    """a: BF16 [M, G, a_width], b: BF16 [M, G, b_width] or None -> (codes [M, G*128], scales), and with
+    want_amax a third item: the groups' amax in the scales' layout."""
     M, G, aw = a.shape
     bw = 0 if b is None else b.shape[-1]
     codes = torch.empty((M, G * 128), dtype=torch.uint8, device=a.device)
@@ -214,15 +228,18 @@ def cat_rotate_fp8(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 12
     else:
         ld = M if scale_ld is None else scale_ld
         scales = torch.empty((G, ld), dtype=torch.float32, device=a.device)
+    amax = torch.empty_like(scales) if want_amax else None
     hq_cat_rotate_fp8(a, a.stride(0), aw, b, 0 if b is None else b.stride(0), bw, M, G, hadamard_n, codes,
-                      scales, scale_layout, ld, stream)
-    return codes, scales
+                      scales, scale_layout, ld, amax, stream)
+    return (codes, scales, amax) if want_amax else (codes, scales)
 
 
-def swiglu_fp8_k128(mode: int, inp: torch.Tensor, K_out: int, stream=None):
-    """K128 FP8 quantization (modes HQ_ACT_*) -> (codes [M, K_out], scales [M, K_out/128])."""
+def swiglu_fp8_k128(mode: int, inp: torch.Tensor, K_out: int, want_amax: bool = False, stream=None):
+    """K128 FP8 quantization (modes HQ_ACT_*) -> (codes [M, K_out], scales [M, K_out/128]), and with
+    want_amax a third item: the groups' amax [M, K_out/128]."""
     M = inp.shape[0]
     codes = torch.empty((M, K_out), dtype=torch.uint8, device=inp.device)
     scales = torch.empty((M, K_out // 128), dtype=torch.float32, device=inp.device)
-    hq_swiglu_fp8_k128(mode, inp, M, K_out, codes, scales, stream)
-    return codes, scales
+    amax = torch.empty_like(scales) if want_amax else None
+    hq_swiglu_fp8_k128(mode, inp, M, K_out, codes, scales, amax, stream)
+    return (codes, scales, amax) if want_amax else (codes, scales)

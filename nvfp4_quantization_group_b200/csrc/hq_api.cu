@@ -130,9 +130,10 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
                              uint8_t* col_codes, uint8_t* col_sf, float* amax_row, float* amax_col,
                              float* sdec_row, float* sdec_col, void* ws, size_t ws_bytes, void* stream) {
     // ---- argument checks (nothing is launched on failure)
-    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
     const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
     if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_ROW_RHT) && !do_row) return HQ_ERR_UNSUPPORTED;
     if (!split_rows || !ws) return HQ_ERR_NULL;
     // code and block-scale buffers are empty (and may be NULL) when M == 0
     if (do_row && (!amax_row || !sdec_row || (M > 0 && (!row_codes || !row_sf)))) return HQ_ERR_NULL;
@@ -168,7 +169,7 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     p.ws = static_cast<uint32_t*>(ws);
     p.S = S;
     p.sign_mask = sign_mask;
-    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE);
+    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT);
     p.col_tiles = (int)(K / NV_TILE);
     int row0 = 0;
     int live[HQ_MAX_SECTIONS];
@@ -241,9 +242,12 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     return launch(pc, nc);
 }
 
+size_t hq_cat_rotate_fp8_workspace_size(void) { return 0; }
+size_t hq_swiglu_fp8_k128_workspace_size(void) { return 0; }
+
 hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, const void* b,
                             int64_t b_row_stride, int b_width, int64_t M, int G, int hadamard_n,
-                            uint8_t* out_fp8, float* scales, int scale_layout, int64_t scale_ld,
+                            uint8_t* out_fp8, float* scales, int scale_layout, int64_t scale_ld, float* amax_opt,
                             void* ws, size_t ws_bytes, void* stream) {
     (void)ws;
     (void)ws_bytes;
@@ -256,7 +260,8 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     if (a_row_stride < (int64_t)G * a_width || (b_width > 0 && b_row_stride < (int64_t)G * b_width))
         return HQ_ERR_SHAPE;
     if (scale_layout == HQ_SCALE_TRANSPOSED && scale_ld < M) return HQ_ERR_SHAPE;
-    if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out_fp8) || !aligned4(scales))
+    if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out_fp8) || !aligned4(scales) ||
+        !aligned4(amax_opt))
         return HQ_ERR_ALIGN;
     const DeviceInfo* dev = device_info();
     if (!dev) return HQ_ERR_CUDA;
@@ -274,6 +279,7 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     p.rotate = hadamard_n == 128;
     p.out = out_fp8;
     p.scales = scales;
+    p.amax = amax_opt;
     p.scale_layout = scale_layout;
     p.scale_ld = scale_ld;
     p.wide = a_width % 16 == 0 && b_width % 16 == 0 && a_row_stride % 16 == 0 && b_row_stride % 16 == 0 &&
@@ -290,7 +296,7 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
 }
 
 hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out, uint8_t* out_fp8,
-                             float* scales, void* ws, size_t ws_bytes, void* stream) {
+                             float* scales, float* amax_opt, void* ws, size_t ws_bytes, void* stream) {
     (void)ws;
     (void)ws_bytes;
     if (mode != HQ_ACT_NONE_BF16 && mode != HQ_ACT_NONE_F32 && mode != HQ_ACT_SWIGLU_F32) return HQ_ERR_UNSUPPORTED;
@@ -298,7 +304,7 @@ hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out,
     if (K_out % 128) return HQ_ERR_ALIGN;
     if (M == 0) return HQ_OK;
     if (!in || !out_fp8 || !scales) return HQ_ERR_NULL;
-    if (!aligned16(in) || !aligned16(out_fp8) || !aligned4(scales)) return HQ_ERR_ALIGN;
+    if (!aligned16(in) || !aligned16(out_fp8) || !aligned4(scales) || !aligned4(amax_opt)) return HQ_ERR_ALIGN;
     const DeviceInfo* dev = device_info();
     if (!dev) return HQ_ERR_CUDA;
     K128Params p;
@@ -309,6 +315,7 @@ hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out,
     p.gpr_magic = 0xFFFFFFFFu / (uint32_t)(K_out / 128);
     p.out = out_fp8;
     p.scales = scales;
+    p.amax = amax_opt;
     constexpr int warps_per_block = K128_THREADS / 32;
     const int64_t pairs = (p.ngroups + 1) / 2;
     const int64_t per_block = (int64_t)warps_per_block * K128_UNROLL;

@@ -264,10 +264,9 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_fp8_kerne
             const uint4 out = *reinterpret_cast<const uint4*>(&sh.codes[k][4 * j]);
             *reinterpret_cast<uint4*>(p.out + v * 128 + 16 * j) = out;
             if (j == 0) {
-                if (p.scale_layout == 0)
-                    p.scales[v] = sc;
-                else
-                    p.scales[(int64_t)cv.g * p.scale_ld + cv.t] = sc;
+                const int64_t si = p.scale_layout == 0 ? v : (int64_t)cv.g * p.scale_ld + cv.t;
+                p.scales[si] = sc;
+                if (p.amax) p.amax[si] = amax;
             }
         }
         __syncwarp();  // the exchange buffers are reused by the next tile
@@ -285,7 +284,9 @@ template <int MODE> struct K128Raw;
 template <> struct K128Raw<HQ_ACT_NONE_BF16> { static constexpr int U = 4; uint4 w[U]; };
 template <> struct K128Raw<HQ_ACT_NONE_F32> { static constexpr int U = 2; uint4 w[U][2]; };
 
-// Scale, codes and the stores of one group whose negated values are ny.
+// Scale, codes and the stores of one group whose negated values are ny
+// (AMAX: the group's amax too).
+template <bool AMAX>
 __device__ __forceinline__ void k128_finish(const K128Params& p, uint32_t g, bool valid, int l, const f2 (&ny)[4],
                                             bool split_store) {
     float m = 0.0f;
@@ -307,11 +308,14 @@ __device__ __forceinline__ void k128_finish(const K128Params& p, uint32_t g, boo
             *reinterpret_cast<uint32_t*>(out + 4 * l) = c.x;
             *reinterpret_cast<uint32_t*>(out + 64 + 4 * l) = c.y;
         }
-        if (l == 0) p.scales[g] = s;
+        if (l == 0) {
+            p.scales[g] = s;
+            if (AMAX) p.amax[g] = m;
+        }
     }
 }
 
-template <int MODE>
+template <int MODE, bool AMAX>
 __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
     const int lane = threadIdx.x & 31;
     const int half = lane >> 4, l = lane & 15;
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
                     ny[2] = pack2(-__uint_as_float(w1.x), -__uint_as_float(w1.y));
                     ny[3] = pack2(-__uint_as_float(w1.z), -__uint_as_float(w1.w));
                 }
-                k128_finish(p, g, ok, l, ny, MODE != HQ_ACT_NONE_BF16);
+                k128_finish<AMAX>(p, g, ok, l, ny, MODE != HQ_ACT_NONE_BF16);
             }
         };
         Raw r0, r1;
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
 #pragma unroll
             for (int u = 0; u < K128_UNROLL; ++u) {
                 const uint32_t g = (base + u) * 2 + half;
-                k128_finish(p, g, base + u < npairs && g < ngroups, l, ny[u], true);
+                k128_finish<AMAX>(p, g, base + u < npairs && g < ngroups, l, ny[u], true);
             }
         }
     }
@@ -436,12 +440,21 @@ void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st) {
     cat_rotate_fp8_kernel<<<grid, CAT_THREADS, 0, st>>>(p);
 }
 
-void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st) {
+template <bool AMAX>
+static void launch_k128_mode(int mode, const K128Params& p, int grid, cudaStream_t st) {
     switch (mode) {
-        case HQ_ACT_NONE_BF16: k128_fp8_kernel<HQ_ACT_NONE_BF16><<<grid, K128_THREADS, 0, st>>>(p); break;
-        case HQ_ACT_NONE_F32: k128_fp8_kernel<HQ_ACT_NONE_F32><<<grid, K128_THREADS, 0, st>>>(p); break;
-        default: k128_fp8_kernel<HQ_ACT_SWIGLU_F32><<<grid, K128_THREADS, 0, st>>>(p); break;
+        case HQ_ACT_NONE_BF16: k128_fp8_kernel<HQ_ACT_NONE_BF16, AMAX><<<grid, K128_THREADS, 0, st>>>(p); break;
+        case HQ_ACT_NONE_F32: k128_fp8_kernel<HQ_ACT_NONE_F32, AMAX><<<grid, K128_THREADS, 0, st>>>(p); break;
+        default: k128_fp8_kernel<HQ_ACT_SWIGLU_F32, AMAX><<<grid, K128_THREADS, 0, st>>>(p); break;
     }
+}
+
+void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st) {
+    // the amax store is a separate instance: the plain kernels keep their registers
+    if (p.amax)
+        launch_k128_mode<true>(mode, p, grid, st);
+    else
+        launch_k128_mode<false>(mode, p, grid, st);
 }
 
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st) {

@@ -27,6 +27,7 @@ struct CatRotateParams {
     int rotate;    // 1: H128 / sqrt(128); 0: none
     uint8_t* out;
     float* scales;
+    float* amax;  // NULL or per-group amax, in the scales' layout
     int scale_layout;
     int64_t scale_ld;
 };
@@ -38,6 +39,7 @@ struct K128Params {
     uint32_t gpr_magic;  // floor((2^32 - 1) / (K_out / 128)): row of a group by multiply-high
     uint8_t* out;
     float* scales;
+    float* amax;  // NULL or per-group amax [M, K_out / 128]
 };
 
 constexpr int K128_THREADS = 256;   // 8 warps, two K128 groups per warp step

@@ -54,9 +54,12 @@ constexpr int NCW = NV_CONSUMER_WARPS;
 constexpr int NST = NV_STAGES;
 constexpr int TILE_BYTES = NV_TILE * NV_TILE * 2;
 
-// header flags; H_SLOW_R / H_SLOW_C: the section encode scale is outside
-// [2^-100, 2^100], where the per-block division takes the slow exact path
-constexpr uint32_t H_VALID = 1u, H_CAST = 2u, H_GAVE_UP = 4u, H_FOLD = 8u, H_SLOW_R = 16u, H_SLOW_C = 32u;
+// header flags; H_SLOW_R / H_SLOW_C: the numerator of the per-block encode
+// factor is outside [2^-100, 2^100], where the division takes the slow exact
+// path; H_FOLD / H_FOLD_R: 0.25 is folded into the columnwise / rotated
+// rowwise encode factors
+constexpr uint32_t H_VALID = 1u, H_CAST = 2u, H_GAVE_UP = 4u, H_FOLD = 8u, H_SLOW_R = 16u, H_SLOW_C = 32u,
+                   H_FOLD_R = 64u;
 
 struct alignas(16) StageHdr {  // 48 bytes, moved as three 16-byte words
     int64_t row0;      // first global row of the tile
@@ -128,11 +131,9 @@ __device__ __forceinline__ void rht_stage1(uint32_t wi, uint32_t wj, bf16_t si, 
     oj = pack2(fma_bf16(xi0, si, -b0), fma_bf16(xi1, si, -b1));
 }
 
-// Unnormalised column RHT, H16 diag(sigma), of a BF16 column pair (16 rows):
-// two columns per packed f32x2 lane; stages 1, 2, 4, 8 in ascending order.
-__device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t (&sg)[16], f2 (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) rht_stage1(w[i], w[i + 1], sg[i], sg[i + 1], v[i], v[i + 1]);
+// Butterfly stages 2, 4, 8 of the 16-point transform, in ascending order, on
+// two independent vectors (the two halves of each packed lane).
+__device__ __forceinline__ void rht_stages(f2 (&v)[16]) {
 #pragma unroll
     for (int h = 2; h < 16; h <<= 1) {
 #pragma unroll
@@ -144,6 +145,32 @@ __device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t
             }
         }
     }
+}
+
+// Unnormalised column RHT, H16 diag(sigma), of a BF16 column pair (16 rows):
+// two columns per packed f32x2 lane; stages 1, 2, 4, 8 in ascending order.
+__device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t (&sg)[16], f2 (&v)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) rht_stage1(w[i], w[i + 1], sg[i], sg[i + 1], v[i], v[i + 1]);
+    rht_stages(v);
+}
+
+// Unnormalised RHT along K of one 16-column block of two rows a and b (word c
+// holds elements 2c, 2c + 1, the even one in the low half): v[i] = {a_i, b_i}
+// of the output.  Stage 1 pairs the two halves of a word, with the signs
+// folded in as in rht_stage1.
+__device__ __forceinline__ void row_rht(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const bf16_t (&sg)[16],
+                                        f2 (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        bf16_t a0, a1, b0, b1;
+        split_bf16x2(wa[c], a0, a1);
+        split_bf16x2(wb[c], b0, b1);
+        const float pa = fma_bf16(a1, sg[2 * c + 1], -0.0f), pb = fma_bf16(b1, sg[2 * c + 1], -0.0f);
+        v[2 * c] = pack2(fma_bf16(a0, sg[2 * c], pa), fma_bf16(b0, sg[2 * c], pb));
+        v[2 * c + 1] = pack2(fma_bf16(a0, sg[2 * c], -pa), fma_bf16(b0, sg[2 * c], -pb));
+    }
+    rht_stages(v);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -247,7 +274,7 @@ struct ProducerState {
     int seg = 0;                // schedule cursor
     int ready_s = -1;           // section whose record is held below
     uint32_t r_fl = 0;          // its header flags (H_FOLD, H_SLOW_*, H_GAVE_UP)
-    float r_sr = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
+    float r_sr = 1.0f, r_srq = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
     uint32_t gave_up = 0;       // sticky once a section wait gave up
     int pf_s = -1;              // section of the prefetched record (lane 0)
     uint64_t pf = 0;
@@ -267,7 +294,7 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
             // ---- the section's record: prefetched one fill ahead, normally
             // already written; else wait (bounded) for it
             uint32_t f = 0u;
-            float sr = 1.0f, sc = 1.0f, scq = 1.0f;
+            float sr = 1.0f, srq = 1.0f, sc = 1.0f, scq = 1.0f;
             if (lane == 0) {
                 const uint64_t* rec_ws = section_records(p) + t.s;
                 uint64_t rec = ps.pf_s == t.s ? ps.pf : ld_relaxed_u64(rec_ws);
@@ -291,15 +318,25 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
                     sr = __uint_as_float((uint32_t)rec & 0x7FFFFFFFu);
                     sc = __uint_as_float((uint32_t)(rec >> 32) & 0x7FFFFFFFu);
                     scq = sc;
+                    srq = sr;
                     if (rec >> 63) {
                         f |= H_FOLD;
                         scq = __fmul_rn(sc, 0.25f);  // exact: sc is in [2^-89, 2^111]
                     }
-                    if (slow_scale(sr)) f |= H_SLOW_R;
+                    // rotated rows: sr in [2^-88, 2^111] implies (sr = RN(2688 /
+                    // A) is monotone) A in [2^-100, 2^100], the range in which
+                    // the fold is exact; sr = 1 (A zero or not finite) folds
+                    // exactly as well
+                    if ((p.flags & HQ_ROW_RHT) && sr >= 0x1p-88f && sr <= 0x1p111f) {
+                        f |= H_FOLD_R;
+                        srq = __fmul_rn(sr, 0.25f);
+                    }
+                    if (slow_scale(srq)) f |= H_SLOW_R;
                     if (slow_scale(scq)) f |= H_SLOW_C;
                 }
             }
             ps.r_sr = __shfl_sync(0xFFFFFFFFu, sr, 0);
+            ps.r_srq = __shfl_sync(0xFFFFFFFFu, srq, 0);
             ps.r_sc = __shfl_sync(0xFFFFFFFFu, sc, 0);
             ps.r_scq = __shfl_sync(0xFFFFFFFFu, scq, 0);
             ps.r_fl = __shfl_sync(0xFFFFFFFFu, f, 0);
@@ -375,7 +412,7 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const uint32_t code = (uint32_t)lane + 32u * m;
-                sh.enc[st][0][code] = block_enc(sh, code, ps.r_sr, fl & H_SLOW_R);
+                sh.enc[st][0][code] = block_enc(sh, code, ps.r_srq, fl & H_SLOW_R);
                 sh.enc[st][1][code] = block_enc(sh, code, ps.r_scq, fl & H_SLOW_C);
             }
             sh.enc_section[st] = t.s;
@@ -405,6 +442,8 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
 }
 
 // ------------------------------------------------------------ compute warps
+// RowRht: the rowwise blocks are rotated along K before their amax and cast.
+template <bool RowRht>
 __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, const uint8_t* tiles, int w,
                                             int lane) {
     uint32_t* const err = p.ws + 2;
@@ -414,6 +453,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
     uint32_t* const done_ws = amax_col_ws + p.S;
     const bool do_row = p.flags & HQ_ROWWISE, do_col = p.flags & HQ_COLWISE;
 
+    const uint8_t* T_cur = tiles;  // the buffer being worked on
     bf16_t sg[16];  // sigma_i as BF16 +-1
 #pragma unroll
     for (int i = 0; i < 16; ++i) sg[i] = ((p.sign_mask >> i) & 1u) ? (bf16_t)0xBF80u : (bf16_t)0x3F80u;
@@ -431,6 +471,19 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         uint32_t coff;     // columnwise: pair 4 vw + jw, row 16 rb
         int cpair;         //   first of its two columns, inside the tile
         uint64_t rs_off0;  // row rr's block-scale offset (+ 4 K16 for rr + 4; codes at 8x)
+    };
+    // This lane's two rows (rr, rr + 4) of part pt in element order: lanes with
+    // `swap` loaded the odd chunk first.
+    auto load_row_pair = [&](const Part& pt, uint32_t (&wa)[8], uint32_t (&wb)[8]) {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const uint32_t ro = pt.roff0 + 4096u * kk;
+            const uint4 lo = *reinterpret_cast<const uint4*>(T_cur + ro);
+            const uint4 hi = *reinterpret_cast<const uint4*>(T_cur + (ro + pt.roff2));
+            const uint32_t wd[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) (kk ? wb : wa)[c] = swap ? wd[c ^ 4] : wd[c];
+        }
     };
     auto part = [&](int vw) {
         Part q;
@@ -464,16 +517,26 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         }
         if (!(h.flags & H_VALID)) break;
         const uint8_t* T = tiles + (size_t)st * TILE_BYTES;
+        T_cur = T;
 
         if (!(h.flags & H_CAST)) {
             // ===================================================== amax tile
             uint32_t mrow = 0u;
-            float mcol = 0.0f;
+            float mrf = 0.0f, mcol = 0.0f;
 #pragma unroll
             for (int pi = 0; pi < 16 / NCW; ++pi) {
             const int vw = w + pi * NCW;
             const Part pt = part(vw);
-            if (do_row) {
+            if (do_row && RowRht) {
+                uint32_t wa[8], wb[8];
+                load_row_pair(pt, wa, wb);
+                f2 v[16];
+                row_rht(wa, wb, sg, v);
+                float r0[16], r1[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) unpack2(v[i], r0[i], r1[i]);
+                mrf = max3(mrf, absmax16(r0), absmax16(r1));
+            } else if (do_row) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const uint32_t ro = pt.roff0 + 4096u * kk;
@@ -496,6 +559,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 mcol = max3(mcol, absmax16(c0), absmax16(c1));
             }
             }  // parts
+            // rotated rows: the maximum of |0.25 y| as binary32 bits (>= 0:
+            // integer order)
+            if (RowRht) mrow = __float_as_uint(__fmul_rn(mrf, 0.25f));
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) {
                 mrow = max(mrow, __shfl_xor_sync(0xFFFFFFFFu, mrow, o));
@@ -534,7 +600,35 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             for (int pi = 0; pi < 16 / NCW; ++pi) {
             const int vw = w + pi * NCW;
             const Part pt = part(vw);
-            if (do_row) {
+            if (do_row && RowRht) {
+                uint32_t wa[8], wb[8];
+                load_row_pair(pt, wa, wb);
+                f2 v[16];
+                row_rht(wa, wb, sg, v);
+                float r0[16], r1[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) unpack2(v[i], r0[i], r1[i]);
+                const uint32_t sf0 = block_sf(__fmul_rn(absmax16(r0), 0.25f), h.senc_r);
+                const uint32_t sf1 = block_sf(__fmul_rn(absmax16(r1), 0.25f), h.senc_r);
+                const f2 e2 = pack2(sh.enc[st][0][sf0], sh.enc[st][0][sf1]);
+                if (!(h.flags & H_FOLD_R)) {
+                    const f2 quarter = pack2(0.25f, 0.25f);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = mul2(v[i], quarter);
+                }
+                float q0[16], q1[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) unpack2(mul2(v[i], e2), q0[i], q1[i]);
+                // rows rr and rr + 4: codes in element order (no chunk swap)
+                *reinterpret_cast<uint2*>(rc_base + 8u * pt.rs_off0) =
+                    make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
+                               e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
+                *reinterpret_cast<uint2*>(rc_base + 8u * (pt.rs_off0 + 4u * K16)) =
+                    make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
+                               e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
+                rs_base[pt.rs_off0] = (uint8_t)sf0;
+                rs_base[pt.rs_off0 + 4u * K16] = (uint8_t)sf1;
+            } else if (do_row) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const uint32_t ro = pt.roff0 + 4096u * kk;
@@ -606,6 +700,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
 }  // namespace
 
+template <bool RowRht>
 __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel(const __grid_constant__ NvParams p) {
     extern __shared__ __align__(1024) uint8_t nv_smem_raw[];
     uint8_t* const nv_smem = nv_smem_raw + ((1024u - (smem_u32(nv_smem_raw) & 1023u)) & 1023u);
@@ -653,7 +748,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
             mbar_wait_bounded(&sh.full[st], last_use & 1u, MBAR_LIMIT);
         }
     } else {
-        nv_consumer(p, sh, nv_smem, warp, lane);
+        nv_consumer<RowRht>(p, sh, nv_smem, warp, lane);
     }
 
     // ---- the last CTA to leave publishes the section scales and resets the
@@ -692,9 +787,13 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
 }
 
 int nvfp4_blocks_per_sm() {
-    int n = 0;
-    cudaFuncSetAttribute(nvfp4_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4_group_kernel, NV_THREADS, NV_DYN_SMEM);
+    // both variants: the grid is sized for the one with fewer resident CTAs
+    int n0 = 0, n1 = 0;
+    cudaFuncSetAttribute(nvfp4_group_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
+    cudaFuncSetAttribute(nvfp4_group_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, nvfp4_group_kernel<false>, NV_THREADS, NV_DYN_SMEM);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, nvfp4_group_kernel<true>, NV_THREADS, NV_DYN_SMEM);
+    const int n = n0 < n1 ? n0 : n1;
     return n > 0 ? n : 1;
 }
 
@@ -705,6 +804,9 @@ int nvfp4_blocks_per_sm() {
 int nvfp4_tiles_in_flight_per_cta() { return NST + 1; }
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
-    nvfp4_group_kernel<<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+    if (p.flags & HQ_ROW_RHT)
+        nvfp4_group_kernel<true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+    else
+        nvfp4_group_kernel<false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
 }
 }  // namespace hq

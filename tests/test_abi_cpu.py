@@ -69,6 +69,7 @@ def _grp(L, x=FAKE, M=256, K=256, splits=(128, 128), flags=3, ptrs=FAKE, ws=FAKE
 def test_group_rht_quant_argument_errors(L):
     assert _grp(L, flags=0) == hq.HQ_ERR_UNSUPPORTED
     assert _grp(L, flags=16) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_RHT) == hq.HQ_ERR_UNSUPPORTED  # rotation without rows
     assert _grp(L, x=0) == hq.HQ_ERR_NULL
     assert _grp(L, ws=0) == hq.HQ_ERR_NULL
     assert _grp(L, ptrs=0) == hq.HQ_ERR_NULL
@@ -84,9 +85,9 @@ def test_group_rht_quant_argument_errors(L):
 
 def test_cat_rotate_fp8_argument_errors(L):
     def call(a=FAKE, a_rs=64 * 64, aw=64, b=FAKE, b_rs=64 * 64, bw=64, M=16, G=64, hn=128, out=FAKE,
-             sc=FAKE, layout=0, ld=16):
+             sc=FAKE, layout=0, ld=16, amax=None):
         return L.hq_cat_rotate_fp8(P(a), a_rs, aw, P(b), b_rs, bw, M, G, hn, P(out), P(sc), layout, ld,
-                                   None, 0, None)
+                                   P(amax), None, 0, None)
     assert call(hn=64) == hq.HQ_ERR_UNSUPPORTED
     assert call(layout=2) == hq.HQ_ERR_UNSUPPORTED
     assert call(aw=64, bw=32) == hq.HQ_ERR_SHAPE                  # widths must sum to 128
@@ -98,11 +99,13 @@ def test_cat_rotate_fp8_argument_errors(L):
     assert call(a_rs=64) == hq.HQ_ERR_SHAPE                        # stride shorter than G groups
     assert call(layout=1, ld=8) == hq.HQ_ERR_SHAPE                 # transposed ld < M
     assert call(out=FAKE + 1) == hq.HQ_ERR_ALIGN
+    assert call(amax=FAKE + 2) == hq.HQ_ERR_ALIGN
+    assert L.hq_cat_rotate_fp8_workspace_size() == 0
 
 
 def test_swiglu_fp8_k128_argument_errors(L):
-    def call(mode=0, inp=FAKE, M=4, K=256, out=FAKE, sc=FAKE):
-        return L.hq_swiglu_fp8_k128(mode, P(inp), M, K, P(out), P(sc), None, 0, None)
+    def call(mode=0, inp=FAKE, M=4, K=256, out=FAKE, sc=FAKE, amax=None):
+        return L.hq_swiglu_fp8_k128(mode, P(inp), M, K, P(out), P(sc), P(amax), None, 0, None)
     assert call(mode=3) == hq.HQ_ERR_UNSUPPORTED
     assert call(K=200) == hq.HQ_ERR_ALIGN
     assert call(M=-1) == hq.HQ_ERR_SHAPE
@@ -110,6 +113,8 @@ def test_swiglu_fp8_k128_argument_errors(L):
     assert call(inp=0) == hq.HQ_ERR_NULL
     assert call(inp=FAKE + 8) == hq.HQ_ERR_ALIGN
     assert call(sc=FAKE + 2) == hq.HQ_ERR_ALIGN
+    assert call(amax=FAKE + 1) == hq.HQ_ERR_ALIGN
+    assert L.hq_swiglu_fp8_k128_workspace_size() == 0
 
 
 def test_convert_and_workspace_argument_errors(L):

@@ -26,14 +26,16 @@ def _dev(a: np.ndarray) -> torch.Tensor:
 def _cat_case(hq, pe, nope, M, G, hadamard_n, layout, ld=None):
     a = _dev(pe)
     b = None if nope is None else _dev(nope)
-    codes, scales = hq.cat_rotate_fp8(a, b, hadamard_n, layout, ld)
+    codes, scales, amax = hq.cat_rotate_fp8(a, b, hadamard_n, layout, ld, want_amax=True)
     torch.cuda.synchronize()
-    want_c, want_s, _ = oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, scale_layout=layout,
-                                              scale_ld=ld if layout else None)
-    got_s = scales.cpu().numpy()
+    want_c, want_s, _, want_a = oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, scale_layout=layout,
+                                                      scale_ld=ld if layout else None, want_amax=True)
+    got_s, got_a = scales.cpu().numpy(), amax.cpu().numpy()
     if layout == oracle.TRANSPOSED:
         got_s, want_s = got_s[:, :M], want_s[:, :M]
+        got_a, want_a = got_a[:, :M], want_a[:, :M]
     assert_bits_equal(got_s, want_s, "scales")
+    assert_bits_equal(got_a, want_a, "amax")
     assert_fp8_codes(codes.cpu().numpy(), want_c,
                      lambda: oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, want_pre=True)[2])
 
@@ -90,10 +92,11 @@ def test_dsa_indexer_full_4096x64(hq):
 
 # ------------------------------------------------------------------ K128
 def _k128_case(hq, mode, x, M, K_out):
-    codes, scales = hq.swiglu_fp8_k128(mode, _dev(x), K_out)
+    codes, scales, amax = hq.swiglu_fp8_k128(mode, _dev(x), K_out, want_amax=True)
     torch.cuda.synchronize()
-    want_c, want_s, _ = oracle.swiglu_fp8_k128(mode, x, M, K_out)
+    want_c, want_s, _, want_a = oracle.swiglu_fp8_k128(mode, x, M, K_out, want_amax=True)
     assert_bits_equal(scales.cpu().numpy(), want_s, "scales")
+    assert_bits_equal(amax.cpu().numpy(), want_a, "amax")
     assert_fp8_codes(codes.cpu().numpy(), want_c, lambda: oracle.swiglu_fp8_k128(mode, x, M, K_out, True)[2])
 
 
@@ -135,9 +138,10 @@ def test_k128_nan_and_inf_groups(hq):
     x = S.normal_f32(331, (2, 128))
     x[0, 3] = np.nan
     x[1, 4] = np.inf
-    codes, scales = hq.swiglu_fp8_k128(hq.HQ_ACT_NONE_F32, _dev(x), 128)
-    want_c, want_s, _ = oracle.swiglu_fp8_k128(oracle.NONE_F32, x, 2, 128)
+    codes, scales, amax = hq.swiglu_fp8_k128(hq.HQ_ACT_NONE_F32, _dev(x), 128, want_amax=True)
+    want_c, want_s, _, want_a = oracle.swiglu_fp8_k128(oracle.NONE_F32, x, 2, 128, want_amax=True)
     assert_bits_equal(scales.cpu().numpy(), want_s, "scales")
+    assert_bits_equal(amax.cpu().numpy(), want_a, "amax")
     assert_fp8_codes(codes.cpu().numpy(), want_c)
     assert (codes[0, 3].item() & 0x7F) == 0x7F
 

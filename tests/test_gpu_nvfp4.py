@@ -157,6 +157,34 @@ def test_extreme_magnitudes(hq):
     _check(got, oracle.group_rht_quant(x, splits, 0x8001, 3), x, splits, 0x8001, 3)
 
 
+@pytest.mark.parametrize("flags", [1 | 4, 1 | 2 | 4, 1 | 2 | 4 | 8])
+def test_row_rht_small_sections(hq, flags):
+    """Rowwise blocks rotated along K: both schedules, with and without the
+    columnwise output."""
+    splits = [128, 0, 256, 128, 0, 384]
+    x = _case(471, 384, splits)
+    mask = 0x9C3A
+    base = flags & 7
+    got, _ = _run(hq, x, splits, mask, flags)
+    _check(got, oracle.group_rht_quant(x, splits, mask, base), x, splits, mask, base)
+    if not flags & 2:
+        assert set(got) == set(ROW_KEYS)
+
+
+@pytest.mark.parametrize("factor", [1e-33, 1e-30, 1e30, 1e33])
+def test_row_rht_scale_range(hq, factor):
+    """Sections on both sides of the range in which 0.25 folds into the
+    rotated rows' encode factors, next to a section of zeros."""
+    splits = [128, 128, 128]
+    xf = S.bf16_bits_to_f32(S.normal_bf16(481, (384, 256))).copy()
+    xf[:128] *= np.float32(factor)
+    xf[128:256] = 0.0
+    xf[256:, 16:32] = 0.0
+    x = S.f32_to_bf16_bits(xf)
+    got, _ = _run(hq, x, splits, 0x00F1, 7)
+    _check(got, oracle.group_rht_quant(x, splits, 0x00F1, 7), x, splits, 0x00F1, 7)
+
+
 @pytest.mark.slow
 def test_dense_nvfp4_8192x4096(hq):
     seed = S.SEEDS["dense_nvfp4"]
@@ -167,13 +195,14 @@ def test_dense_nvfp4_8192x4096(hq):
 
 
 @pytest.mark.slow
-def test_grouped_moe_16384x7168(hq):
+@pytest.mark.parametrize("flags", [3, 7])
+def test_grouped_moe_16384x7168(hq, flags):
     seed = S.SEEDS["grouped_moe"]
     x = S.normal_bf16(seed, (16384, 7168))
     splits = S.moe_splits(seed)
     mask = S.sign_mask16(seed)
-    got, _ = _run(hq, x, splits, mask, 3)
-    _check(got, oracle.group_rht_quant(x, splits, mask, 3), x, splits, mask, 3)
+    got, _ = _run(hq, x, splits, mask, flags)
+    _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
 
 
 def test_bounded_wait_reports_timeout_and_recovers(hq):
