@@ -173,14 +173,16 @@ def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False, want_amax=False):
     return (out, scales, pre, amax) if want_amax else (out, scales, pre)
 
 
-ROWWISE, COLWISE, ROW_RHT = 1, 2, 4
+ROWWISE, COLWISE, ROW_RHT, AMAX_GIVEN = 1, 2, 4, 16
 
 
-def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=False):
+def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=False, amax_row=None,
+                    amax_col=None):
     """Grouped RHT16 + NVFP4 cast.  x: uint16 BF16 bits [M, K].
 
     ROW_RHT (with ROWWISE) rotates every 16-element row block along K before
-    the rowwise amax and cast.
+    the rowwise amax and cast.  AMAX_GIVEN takes the section amax values from
+    amax_row / amax_col (float [S]) instead of computing them.
 
     Returns a dict with row_codes [M, K/2], row_sf [M, K/16], col_codes
     [M*K/2], col_sf [M*K/16] (sections concatenated, each [K, M_s/...]),
@@ -206,6 +208,11 @@ def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=
         r["sdec_col"] = np.empty(S, dtype=np.float32)
         if want_pre:
             r["col_pre"] = np.empty(M * K, dtype=np.float32)
+    if flags & AMAX_GIVEN:
+        if flags & ROWWISE:
+            r["amax_row"][:] = np.asarray(amax_row, dtype=np.float32)
+        if flags & COLWISE:
+            r["amax_col"][:] = np.asarray(amax_col, dtype=np.float32)
     g = r.get
     rc = lib().hqo_group_rht_quant(_ptr(x), M, K, _ptr(splits), S, sign_mask, flags,
                                    _ptr(g("row_codes")), _ptr(g("row_sf")), _ptr(g("col_codes")),

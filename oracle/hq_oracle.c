@@ -434,8 +434,15 @@ static void rht16(const float *x, uint16_t sign_mask, float *v)
  *   starting at row r0 owns col_codes[K*r0/2 ...] as [K, M_s/2] and
  *   col_sf[K*r0/16 ...] as [K, M_s/16].
  * amax_*[s], sdec_*[s] receive A and 1/S_enc of the requested directions;
- * an empty section gives A = 0, sdec = 1.  row_pre / col_pre, when given,
- * receive the value rounded to E2M1 per element, in the output's layout.
+ * an empty section gives A = 0, sdec = 1.
+ * flags bit 4 (amax given): amax_*[s] are inputs instead, the section amax a
+ *   caller computed beforehand (of the rotated values where the direction is
+ *   rotated); there is no amax pass, S_enc and everything after it follow
+ *   from the given A, and sdec_*[s] = 1/S_enc(A) for every section, empty
+ *   ones included.  The pages do not describe this mode: it is the one-pass
+ *   cast that a known amax allows, checked here by its definition.
+ * row_pre / col_pre, when given, receive the value rounded to E2M1 per
+ * element, in the output's layout.
  */
 int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                         const int64_t *split_rows, int S, uint16_t sign_mask, unsigned flags,
@@ -458,11 +465,12 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
     float blk[16], v[16];
     for (int s = 0; s < S; ++s) {
         const int64_t Ms = split_rows[s];
+        const int given = (flags & 16) != 0;
         if (flags & 1) {
             const int rotate = (flags & 4) != 0;
             /* first pass: section amax (of the rotated blocks if rotating) */
             float A = 0.0f;
-            for (int64_t r = r0; r < r0 + Ms; ++r)
+            for (int64_t r = r0; r < r0 + Ms && !given; ++r)
                 for (int64_t kb = 0; kb < K / 16; ++kb) {
                     for (int i = 0; i < 16; ++i)
                         blk[i] = bf16_value(x[r * K + kb * 16 + i]);
@@ -471,6 +479,8 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                     for (int i = 0; i < 16; ++i)
                         A = fmaxf(A, fabsf(rotate ? v[i] : blk[i]));
                 }
+            if (given)
+                A = amax_row[s];
             float S_enc = global_encode_scale(A);
             amax_row[s] = A;
             sdec_row[s] = 1.0f / S_enc;
@@ -489,7 +499,7 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
         if (flags & 2) {
             /* first pass: section amax of the rotated values */
             float A = 0.0f;
-            for (int64_t c = 0; c < K; ++c)
+            for (int64_t c = 0; c < K && !given; ++c)
                 for (int64_t mb = 0; mb < Ms / 16; ++mb) {
                     for (int i = 0; i < 16; ++i)
                         blk[i] = bf16_value(x[(r0 + mb * 16 + i) * K + c]);
@@ -497,6 +507,8 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                     for (int i = 0; i < 16; ++i)
                         A = fmaxf(A, fabsf(v[i]));
                 }
+            if (given)
+                A = amax_col[s];
             float S_enc = global_encode_scale(A);
             amax_col[s] = A;
             sdec_col[s] = 1.0f / S_enc;
@@ -512,7 +524,7 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                                 col_pre ? col_pre + K * r0 + c * Ms + mb * 16 : 0);
                 }
         }
-        if (Ms == 0) {
+        if (Ms == 0 && !given) {
             if (flags & 1) { amax_row[s] = 0.0f; sdec_row[s] = 1.0f; }
             if (flags & 2) { amax_col[s] = 0.0f; sdec_col[s] = 1.0f; }
         }

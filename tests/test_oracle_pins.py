@@ -526,6 +526,60 @@ def test_nvfp4_row_rht_equals_column_rht_of_transpose():
     assert r["amax_row"][0] == c["amax_col"][0] and r["sdec_row"][0] == c["sdec_col"][0]
 
 
+def test_nvfp4_amax_given_single_pass():
+    """AMAX_GIVEN: the section amax values are inputs.  Given the computed
+    ones, every output equals the two-pass result; given others, the block
+    scales and codes follow the closed-form rule from S_enc = 2688 / A_given
+    (saturating when A_given is below the data's amax), and an empty section
+    keeps its given amax with sdec = 1 / S_enc."""
+    x, splits, mask = _nvfp4_case(seed=87, splits=(128, 0, 256))
+    both = oracle.ROWWISE | oracle.COLWISE
+    ref = oracle.group_rht_quant(x, splits, mask, both)
+    same = oracle.group_rht_quant(x, splits, mask, both | oracle.AMAX_GIVEN,
+                                  amax_row=ref["amax_row"], amax_col=ref["amax_col"])
+    for k in ref:
+        np.testing.assert_array_equal(same[k], ref[k], err_msg=k)
+    rot = oracle.group_rht_quant(x, splits, mask, oracle.ROWWISE | oracle.ROW_RHT)
+    rot2 = oracle.group_rht_quant(x, splits, mask, oracle.ROWWISE | oracle.ROW_RHT | oracle.AMAX_GIVEN,
+                                  amax_row=rot["amax_row"])
+    for k in rot:
+        np.testing.assert_array_equal(rot2[k], rot[k], err_msg=k)
+
+    given = np.array([2.0, 3.0, 0.25], dtype=np.float32) * np.maximum(ref["amax_row"], 1)
+    r = oracle.group_rht_quant(x, splits, mask, oracle.ROWWISE | oracle.AMAX_GIVEN, want_pre=True,
+                               amax_row=given)
+    np.testing.assert_array_equal(r["amax_row"], given)
+    S_encs = [np.float32(2688) / g for g in given]
+    assert r["sdec_row"][1] == np.float32(1) / S_encs[1]          # empty section
+    xf = S.bf16_bits_to_f32(x)
+    M, K = x.shape
+    r0 = 0
+    for s, Ms in enumerate(splits):
+        if Ms == 0:
+            continue
+        blocks = xf[r0:r0 + Ms].reshape(Ms, K // 16, 16)
+        ab = np.max(np.abs(blocks), axis=-1)
+        sf = r["row_sf"][r0:r0 + Ms]
+        for i in range(0, Ms, 29):
+            for kb in range(K // 16):
+                t = frac(ab[i, kb]) / 6 * frac(S_encs[s])
+                want = nearest_code(t, E4C, E4V, 0x80, False)
+                if sf[i, kb] != want:
+                    assert near_midpoint(t, E4V)
+        sff = _e4m3_vals(sf)
+        enc = np.where(sff == 0, 0, S_encs[s] / sff.astype(np.float32)).astype(np.float32)
+        pre = r["row_pre"][r0:r0 + Ms]
+        np.testing.assert_array_equal(pre, (blocks * enc[..., None]).reshape(Ms, K).astype(np.float32))
+        nib = _unpack(r["row_codes"][r0:r0 + Ms])
+        if given[s] < ref["amax_row"][s]:
+            # below the data's amax: the top block scale saturates at 448 and
+            # codes saturate at 6
+            i, kb = np.unravel_index(np.argmax(ab), ab.shape)
+            assert sf[i, kb] == 0x7E
+            assert np.any((nib & 7) == 7)
+        r0 += Ms
+
+
 def test_nvfp4_zero_section_and_tiny_values():
     x = np.zeros((256, 128), dtype=np.uint16)
     x[128:] = S.normal_bf16(97, (128, 128))
