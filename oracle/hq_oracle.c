@@ -376,10 +376,13 @@ int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
  *   code  = e2m1(v_i * enc)
  * so that v_i ~= e2m1_value(code) * float(sf) * sdec.
  */
+/* S_enc = 2688 / A; 1 when A is not positive (0, or a negative or NaN amax
+ * given by the caller: reading, treated like A = 0) or 2688 / A is not
+ * finite. */
 static float global_encode_scale(float A)
 {
     float S = 2688.0f / A;
-    if (A == 0.0f || !isfinite(S))
+    if (!(A > 0.0f) || !isfinite(S))
         S = 1.0f;
     return S;
 }

@@ -578,6 +578,14 @@ def test_nvfp4_amax_given_single_pass():
             assert sf[i, kb] == 0x7E
             assert np.any((nib & 7) == 7)
         r0 += Ms
+    # a given amax that is not positive (negative, NaN) acts like 0: S_enc = 1
+    z = oracle.group_rht_quant(x, splits, mask, both | oracle.AMAX_GIVEN, amax_row=np.zeros(3, np.float32),
+                               amax_col=np.zeros(3, np.float32))
+    assert np.all(z["sdec_row"] == 1) and np.all(z["sdec_col"] == 1)
+    bad = np.array([-1.0, np.nan, -0.0], dtype=np.float32)
+    w = oracle.group_rht_quant(x, splits, mask, both | oracle.AMAX_GIVEN, amax_row=bad, amax_col=bad[::-1])
+    for k in ("row_codes", "row_sf", "col_codes", "col_sf", "sdec_row", "sdec_col"):
+        np.testing.assert_array_equal(w[k], z[k], err_msg=k)
 
 
 def test_nvfp4_zero_section_and_tiny_values():
