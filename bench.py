@@ -54,7 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="grouped_moe",
-                    choices=("grouped_moe", "dense_nvfp4", "dsa_indexer", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
+                    choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4",
+                             "dsa_indexer", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
     ap.add_argument("--no-extras", action="store_true", help="time only the headline workload")
     ap.add_argument("--schedule", choices=("fused", "two_pass"), default="fused")
     ap.add_argument("--no-e2e", action="store_true")
@@ -325,6 +326,67 @@ class GroupedNVFP4(Workload):
                 f"one {rows}-row section of the BF16 [{self.M},{self.K}] input (rows 0..{rows - 1})")
 
 
+class GroupedAmaxGiven(GroupedNVFP4):
+    """The same workload with the section amax values supplied by the caller
+    (HQ_AMAX_GIVEN): one pass over x.  The amax values come from one ordinary
+    call before the timed steps."""
+    name = "grouped_moe_amax_given"
+
+    def setup(self, hq, torch, host):
+        super().setup(hq, torch, host)
+        GroupedNVFP4.call(self, self.dev_in, self.out)   # fills amax_row / amax_col
+        torch.cuda.synchronize()
+
+    def config(self):
+        c = super().config()
+        c["workload"] += ", section amax given (single pass)"
+        c["schedule"] = "amax given"
+        return c
+
+    def call(self, inputs, out):
+        hq = self.hq
+        hq.hq_group_rht_quant(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask,
+                              hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_AMAX_GIVEN,
+                              out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
+                              out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
+
+    def oracle_sample(self, host, rows=512):
+        import oracle
+        x = host["x"][:rows]
+        r = oracle.group_rht_quant(x, [rows], self.mask, oracle.ROWWISE | oracle.COLWISE)
+        flags = oracle.ROWWISE | oracle.COLWISE | oracle.AMAX_GIVEN
+        return (lambda: oracle.group_rht_quant(x, [rows], self.mask, flags, amax_row=r["amax_row"],
+                                               amax_col=r["amax_col"]),
+                rows * self.K * 2 + 2 * (rows * self.K // 2 + rows * self.K // 16),
+                f"one {rows}-row section of the BF16 [{self.M},{self.K}] input, amax given")
+
+
+class GroupedRowRHT(GroupedNVFP4):
+    """The same workload with the rowwise output rotated too (HQ_ROW_RHT)."""
+    name = "grouped_moe_row_rht"
+
+    def config(self):
+        c = super().config()
+        c["workload"] += ", rowwise output rotated too"
+        c["directions"] = "rowwise (RHT16 along K) + columnwise"
+        return c
+
+    def call(self, inputs, out):
+        hq = self.hq
+        flags = hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_ROW_RHT | (0 if self.schedule == "fused" else hq.HQ_TWO_PASS)
+        hq.hq_group_rht_quant(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask, flags,
+                              out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
+                              out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
+
+    def oracle_sample(self, host, rows=512):
+        import oracle
+        x = host["x"][:rows]
+        flags = oracle.ROWWISE | oracle.COLWISE | oracle.ROW_RHT
+        return (lambda: oracle.group_rht_quant(x, [rows], self.mask, flags),
+                rows * self.K * 2 + 2 * (rows * self.K // 2 + rows * self.K // 16),
+                f"one {rows}-row section of the BF16 [{self.M},{self.K}] input, rows rotated too")
+
+
 class DenseNVFP4(GroupedNVFP4):
     name = "dense_nvfp4"
 
@@ -459,6 +521,8 @@ class QMoE(Workload):
 
 def make_workload(name: str, rank: int, schedule: str = "fused") -> Workload:
     return {"grouped_moe": lambda: GroupedNVFP4(rank, schedule=schedule),
+            "grouped_moe_amax_given": lambda: GroupedAmaxGiven(rank),
+            "grouped_moe_row_rht": lambda: GroupedRowRHT(rank, schedule=schedule),
             "dense_nvfp4": lambda: DenseNVFP4(rank, schedule=schedule),
             "dsa_indexer": lambda: DSAIndexer(rank),
             "fp8_single": lambda: FP8Single(rank),
@@ -644,7 +708,8 @@ def run_ours(args, ranks: Ranks) -> None:
         del main, host_main
         torch.cuda.empty_cache()
         extras = {}
-        for name in ("dense_nvfp4", "dsa_indexer", "qmoe_bf16", "qmoe_swiglu", "fp8_single"):
+        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4", "dsa_indexer", "qmoe_bf16",
+                     "qmoe_swiglu", "fp8_single"):
             if name == args.workload:
                 continue
             r = measure(torch, hq, name, args, ranks, flush)

@@ -58,6 +58,8 @@ typedef enum hq_status {
 #define HQ_COLWISE 2u      /* columnwise NVFP4 output (RHT16 along M, transposed) */
 #define HQ_ROW_RHT 4u      /* with HQ_ROWWISE: the rowwise output casts the RHT16
                               of each 16-column block along K instead of x */
+#define HQ_AMAX_GIVEN 16u  /* amax_row / amax_col are inputs: the caller's section
+                              amax values; one pass, no amax computation */
 #define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
                               instead of one launch in which each section's
                               cast follows its amax while the rows are still
@@ -88,10 +90,10 @@ const char *hq_status_string(hq_status s);
 /*
  * Workspace bytes hq_group_rht_quant needs for `num_sections` sections
  * (1 <= num_sections <= HQ_MAX_SECTIONS; 0 otherwise).  The first 4 bytes
- * are the tile-scheduler counter of [GRP]; an error word, per-section amax
- * accumulators, completion counters and 64-bit section ready records (the
- * section encode scales, written once the section's amax is complete)
- * follow.  The size query is the reviewers' proposal in [GRP].
+ * are the tile-scheduler counter of [GRP]; an exit count, an error word, an
+ * abort flag, then per section an amax accumulator per direction and a count
+ * of its completed amax tiles follow (16 + 12 * S bytes, rounded up to 256).
+ * The size query is the reviewers' proposal in [GRP].
  */
 size_t hq_group_rht_quant_workspace_size(int num_sections);
 
@@ -126,12 +128,14 @@ hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *strea
  *             HQ_ROW_RHT, of each 16-column block of a row).
  *  flags      HQ_ROWWISE | HQ_COLWISE (at least one), optionally HQ_ROW_RHT
  *             (only with HQ_ROWWISE; the grouped-quant pages speak of the RHT
- *             on both outputs, their fused kernel rotates only the columns)
- *             and HQ_TWO_PASS.
+ *             on both outputs, their fused kernel rotates only the columns),
+ *             HQ_AMAX_GIVEN and HQ_TWO_PASS (ignored with HQ_AMAX_GIVEN).
  *
  * For section s (rows [r0, r0 + M_s)) and each requested direction:
  *   A_s = max |v| over the section's values (v = x rowwise, the RHT16 output
- *   along K with HQ_ROW_RHT; v = RHT16 output columnwise), S_enc = 2688 / A_s (1 when A_s == 0 or not finite),
+ *   along K with HQ_ROW_RHT; v = RHT16 output columnwise), or with
+ *   HQ_AMAX_GIVEN the caller's amax_*[s]; S_enc = 2688 / A_s (1 when A_s is
+ *   not positive or the quotient is not finite),
  *   sdec = 1 / S_enc; for each block of 16 values along the quantized
  *   direction: sf = E4M3((a_b / 6) * S_enc), code_i = E2M1(v_i * S_enc / sf)
  *   (0 when sf == 0); saturating round-to-nearest-even conversions.
@@ -145,6 +149,9 @@ hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *strea
  *  col_sf     uint8 [M*K/16]     per section s: [K, M_s/16] at byte K*r0/16
  *  amax_row, sdec_row  float [S] (HQ_ROWWISE)
  *  amax_col, sdec_col  float [S] (HQ_COLWISE)
+ *  With HQ_AMAX_GIVEN amax_row / amax_col are inputs (device, read only, set
+ *  before the call in stream order) and only sdec_* is written; the call then
+ *  reads x once (the cast pass alone).
  *  Pointers of a direction not requested may be NULL, and so may the code
  *  and block-scale buffers when M == 0.
  *
@@ -171,7 +178,7 @@ hq_status hq_group_rht_quant(const void *x, int64_t M, int64_t K,
  *
  * Arguments, outputs and errors are those of hq_group_rht_quant without
  * ws / ws_bytes.  The scratch words live in a fixed array inside the library
- * (5376 bytes, room for HQ_MAX_SECTIONS = 256 sections; S > 256 returns
+ * (3328 bytes, room for HQ_MAX_SECTIONS = 256 sections; S > 256 returns
  * HQ_ERR_SHAPE), present on every GPU that loads the library until the
  * process exits.  The call allocates nothing: it clears the array with an
  * enqueued memset and launches the kernel.  The first call on a device looks

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libhq.so")
 
 HQ_OK, HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA, \
     HQ_ERR_TIMEOUT = range(8)
-HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS = 1, 2, 4, 8
+HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS, HQ_AMAX_GIVEN = 1, 2, 4, 8, 16
 HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
 HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
 HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1

@@ -45,9 +45,8 @@ inline hq_status launch_status() {
     return cudaPeekAtLastError() == cudaSuccess ? HQ_OK : (cudaGetLastError(), HQ_ERR_CUDA);
 }
 
-// header, amax_row[S], amax_col[S], done[S], then (8-byte aligned) the 64-bit
-// section ready records[S]
-size_t nv_ws_words(int S) { return (((size_t)NV_WS_HEADER + 3 * (size_t)S + 1) & ~(size_t)1) + 2 * (size_t)S; }
+// header, amax_row[S], amax_col[S], done[S] (amax tiles counted per section)
+size_t nv_ws_words(int S) { return (size_t)NV_WS_HEADER + 3 * (size_t)S; }
 
 // The driver's tensor-map encoder, reached once through the runtime (no link
 // against the driver library).
@@ -130,7 +129,7 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
                              uint8_t* col_codes, uint8_t* col_sf, float* amax_row, float* amax_col,
                              float* sdec_row, float* sdec_col, void* ws, size_t ws_bytes, void* stream) {
     // ---- argument checks (nothing is launched on failure)
-    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
     const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
     if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
     if ((flags & HQ_ROW_RHT) && !do_row) return HQ_ERR_UNSUPPORTED;
@@ -169,7 +168,7 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     p.ws = static_cast<uint32_t*>(ws);
     p.S = S;
     p.sign_mask = sign_mask;
-    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT);
+    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN);
     p.col_tiles = (int)(K / NV_TILE);
     int row0 = 0;
     int live[HQ_MAX_SECTIONS];
@@ -200,6 +199,15 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
         return launch_status();
     };
 
+    if (flags & HQ_AMAX_GIVEN) {
+        // One pass: the cast segments alone; each section's record comes from
+        // the caller's amax.
+        uint32_t next = 0;
+        for (int k = 0; k < nlive; ++k) add_seg(p, live[k], 1, next);
+        p.finalize = 1;
+        p.reset_counter = 1;
+        return launch(p, next);
+    }
     if (!(flags & HQ_TWO_PASS)) {
         // One launch.  The cast segment of a section follows its amax segment
         // once `lag` more tiles have been scheduled (the tiles the grid holds

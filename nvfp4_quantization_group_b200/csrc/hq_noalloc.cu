@@ -16,10 +16,11 @@
 namespace {
 
 // Scratch for up to HQ_MAX_SECTIONS (256) sections: the workspace size the
-// grouped call asks for at 256 sections, 5376 bytes, held on every GPU that
+// grouped call asks for at 256 sections (3088 bytes rounded up to 3328, the
+// size the call clears), held on every GPU that
 // loads the library until the process exits.
-constexpr int kNoallocWords = 5376 / 4;
-static_assert(4 * (((hq::NV_WS_HEADER + 3 * HQ_MAX_SECTIONS + 1) & ~1) + 2 * HQ_MAX_SECTIONS) <= 5376,
+constexpr int kNoallocWords = 3328 / 4;
+static_assert(((4 * (hq::NV_WS_HEADER + 3 * HQ_MAX_SECTIONS) + 255) & ~255) <= 3328,
               "scratch too small");
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocWords];
 

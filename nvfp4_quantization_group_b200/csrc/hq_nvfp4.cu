@@ -91,10 +91,12 @@ struct NvShared {
 // swizzle pattern is defined on 1024-byte aligned addresses)
 constexpr int NV_DYN_SMEM = NST * TILE_BYTES + (int)sizeof(NvShared) + 1024;
 
-// Section encode scale: 2688 / A (6 * 448), 1 when A == 0 or not finite.
+// Section encode scale: 2688 / A (6 * 448); 1 when A is not positive (a
+// computed amax is 0 at worst; a given one may be negative or NaN) or the
+// quotient is not finite.
 __device__ __forceinline__ float global_encode(float A) {
     float S = __fdiv_rn(2688.0f, A);
-    if (A == 0.0f || !isfinite(S)) S = 1.0f;
+    if (!(A > 0.0f) || !isfinite(S)) S = 1.0f;
     return S;
 }
 
@@ -230,34 +232,34 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
 
 namespace {
 
-// ------------------------------------------------------ section records
-// A section's ready record (64 bits in the workspace, 0 until the section's
-// amax is complete) carries what its cast tiles need, so reading it is the
-// whole wait: low word senc_r | 1 << 31 (never 0 once written), high word
-// senc_c | fold << 31.  It is written by the compute warp whose amax tile
-// completes the section.
-__device__ __forceinline__ uint64_t* section_records(const NvParams& p) {
-    return reinterpret_cast<uint64_t*>(p.ws + ((NV_WS_HEADER + 3 * p.S + 1) & ~1));
-}
+// ------------------------------------------------------ section completion
+// Compute warps publish an amax tile with reductions that return nothing (the
+// tile's maxima, then a release increment of the section's tile count), so
+// no compute warp waits on a global round trip.  The producer, about to fill
+// a buffer with the section's first cast tile, waits (bounded) until the
+// count reaches the section's amax tiles, then reads the maxima after an
+// acquire fence and derives the section record: low word senc_r, high word
+// senc_c | fold << 31.
 __device__ __forceinline__ uint64_t make_record(float Ar, float Ac) {
     // 0.25 folds into the column encode factor when neither 0.25 y nor
     // 0.25 enc can leave the normal range: A in [2^-100, 2^100]
     const uint32_t fold = (Ac >= 7.8886091e-31f && Ac <= 1.2676506e30f) ? 1u : 0u;
-    return (uint64_t)(__float_as_uint(global_encode(Ar)) | 0x80000000u) |
+    return (uint64_t)__float_as_uint(global_encode(Ar)) |
            ((uint64_t)(__float_as_uint(global_encode(Ac)) | (fold << 31)) << 32);
 }
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* q) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(q) : "memory");
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* q) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(q) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* q, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(q), "l"(v) : "memory");
+// with a relaxed load before it that saw the final count: an acquire pattern
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void red_max_u32(uint32_t* q, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" :: "l"(q), "r"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* q, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(q), "r"(v) : "memory");
-    return old;
+// orders this thread's earlier writes and reductions (the maxima) before it
+__device__ __forceinline__ void red_release_add_u32(uint32_t* q, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(q), "r"(v) : "memory");
 }
 // Per-block encode factor S / value(sf), correctly rounded (0 for codes 0
 // and 127); `slow` when S is outside [2^-100, 2^100].
@@ -276,8 +278,8 @@ struct ProducerState {
     uint32_t r_fl = 0;          // its header flags (H_FOLD, H_SLOW_*, H_GAVE_UP)
     float r_sr = 1.0f, r_srq = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
     uint32_t gave_up = 0;       // sticky once a section wait gave up
-    int pf_s = -1;              // section of the prefetched record (lane 0)
-    uint64_t pf = 0;
+    int pf_s = -1;              // section of the prefetched tile count (lane 0)
+    uint32_t pf = 0;
     TileInfo nt;                // the next fill's tile, decoded one fill ahead
 };
 
@@ -291,31 +293,44 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
     if (t.phase == 1) {
         fl |= H_CAST;
         if (t.s != ps.ready_s) {
-            // ---- the section's record: prefetched one fill ahead, normally
-            // already written; else wait (bounded) for it
+            // ---- the section's scales: from the caller's amax, or once the
+            // section's amax tiles are all counted (the count is prefetched
+            // one fill ahead and normally complete; else wait, bounded)
             uint32_t f = 0u;
             float sr = 1.0f, srq = 1.0f, sc = 1.0f, scq = 1.0f;
             if (lane == 0) {
-                const uint64_t* rec_ws = section_records(p) + t.s;
-                uint64_t rec = ps.pf_s == t.s ? ps.pf : ld_relaxed_u64(rec_ws);
-                uint32_t spins = 0;
+                uint64_t rec = 0u;
                 uint32_t g = ps.gave_up;
-                while (!g && rec == 0u) {
-                    if (*(volatile uint32_t*)abort_flag != 0u) {
-                        g = 1u;
-                    } else if (++spins > SPIN_LIMIT) {
-                        atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
-                        atomicExch(abort_flag, 1u);
-                        g = 1u;
-                    } else {
-                        __nanosleep(64);
-                        rec = ld_relaxed_u64(rec_ws);
+                if (p.flags & HQ_AMAX_GIVEN) {
+                    rec = make_record((p.flags & HQ_ROWWISE) ? p.amax_row[t.s] : 0.0f,
+                                      (p.flags & HQ_COLWISE) ? p.amax_col[t.s] : 0.0f);
+                } else if (!g) {
+                    const uint32_t* const done = p.ws + NV_WS_HEADER + 2 * p.S + t.s;
+                    const uint32_t target = (uint32_t)(t.ms / NV_TILE) * (uint32_t)p.col_tiles;
+                    uint32_t d = ps.pf_s == t.s ? ps.pf : ld_relaxed_u32(done);
+                    uint32_t spins = 0;
+                    while (!g && d < target) {
+                        if (*(volatile uint32_t*)abort_flag != 0u) {
+                            g = 1u;
+                        } else if (++spins > SPIN_LIMIT) {
+                            atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
+                            atomicExch(abort_flag, 1u);
+                            g = 1u;
+                        } else {
+                            __nanosleep(64);
+                            d = ld_relaxed_u32(done);
+                        }
+                    }
+                    if (!g) {
+                        fence_acq_rel_gpu();  // every counted tile's maxima are visible now
+                        rec = make_record(__uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + t.s)),
+                                          __uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + p.S + t.s)));
                     }
                 }
                 if (g) {
                     f |= H_GAVE_UP;
                 } else {
-                    sr = __uint_as_float((uint32_t)rec & 0x7FFFFFFFu);
+                    sr = __uint_as_float((uint32_t)rec);
                     sc = __uint_as_float((uint32_t)(rec >> 32) & 0x7FFFFFFFu);
                     scq = sc;
                     srq = sr;
@@ -377,7 +392,7 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
     // Lane 0 keeps three claims in flight in ca, cb, cc: fill k takes its tile
     // from one register, refills it with a new claim (read three fills
     // later) and looks at the next fill's tile, claimed two fills earlier, to
-    // prefetch that tile's section record.
+    // prefetch its section's amax tile count.
     uint32_t ca = 0, cb = 0, cc = 0;
     if (lane == 0) {
         ca = atomicAdd(counter, 1u);
@@ -425,12 +440,13 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
             tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, t.col0 + 64, c1, 0, &sh.full[st]);
         }
         mbar_arrive(&sh.full[st]);  // every lane: releases the header writes
-        // ---- prefetch the section record of the next fill's tile
+        // ---- prefetch the amax tile count of the next fill's section
         const uint32_t nt = __shfl_sync(0xFFFFFFFFu, next, 0);
         if (nt < total) {
             ps.nt = decode(p, sh, nt, ps.seg);
-            if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s) {
-                ps.pf = ld_relaxed_u64(section_records(p) + ps.nt.s);
+            if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s &&
+                !(p.flags & HQ_AMAX_GIVEN)) {
+                ps.pf = ld_relaxed_u32(p.ws + NV_WS_HEADER + 2 * p.S + ps.nt.s);
                 ps.pf_s = ps.nt.s;
             }
         }
@@ -580,16 +596,10 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     sh.acc_row[st] = 0u;
                     sh.acc_col[st] = 0u;
                     sh.acc_cnt[st] = 0u;
-                    if (do_row) atomicMax(amax_row_ws + h.s, ar);
-                    if (do_col) atomicMax(amax_col_ws + h.s, ac);
-                    // acq_rel: the maxima above are visible first, and the
-                    // tile completing the section sees every tile's maxima
-                    const uint32_t target = (uint32_t)(h.ms / NV_TILE) * (uint32_t)p.col_tiles;
-                    if (atom_add_acq_rel(done_ws + h.s, 1u) == target - 1u) {
-                        const float Ar = __uint_as_float(*(volatile uint32_t*)(amax_row_ws + h.s));
-                        const float Ac = __uint_as_float(*(volatile uint32_t*)(amax_col_ws + h.s));
-                        st_relaxed_u64(section_records(p) + h.s, make_record(Ar, Ac));
-                    }
+                    if (do_row) red_max_u32(amax_row_ws + h.s, ar);
+                    if (do_col) red_max_u32(amax_col_ws + h.s, ac);
+                    // release: a producer that sees the count sees the maxima
+                    red_release_add_u32(done_ws + h.s, 1u);
                 }
             }
         } else if (!(h.flags & H_GAVE_UP)) {
@@ -762,21 +772,21 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
     if (sh.last == 0) return;
     __threadfence();
     if (p.finalize) {
+        const bool given = p.flags & HQ_AMAX_GIVEN;  // amax_* are inputs: only sdec is written
         for (int s = tid; s < p.S; s += NV_THREADS) {
             if (do_row) {
-                const float A = __uint_as_float(*(volatile uint32_t*)(amax_row_ws + s));
-                p.amax_row[s] = A;
+                const float A = given ? p.amax_row[s] : __uint_as_float(*(volatile uint32_t*)(amax_row_ws + s));
+                if (!given) p.amax_row[s] = A;
                 p.sdec_row[s] = __fdiv_rn(1.0f, global_encode(A));
                 amax_row_ws[s] = 0;
             }
             if (do_col) {
-                const float A = __uint_as_float(*(volatile uint32_t*)(amax_col_ws + s));
-                p.amax_col[s] = A;
+                const float A = given ? p.amax_col[s] : __uint_as_float(*(volatile uint32_t*)(amax_col_ws + s));
+                if (!given) p.amax_col[s] = A;
                 p.sdec_col[s] = __fdiv_rn(1.0f, global_encode(A));
                 amax_col_ws[s] = 0;
             }
             done_ws[s] = 0;
-            section_records(p)[s] = 0u;
         }
     }
     if (tid == 0 && p.reset_counter) {

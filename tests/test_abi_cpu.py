@@ -53,6 +53,7 @@ def test_workspace_size_query():
     s1 = hq.hq_group_rht_quant_workspace_size(1)
     s32 = hq.hq_group_rht_quant_workspace_size(32)
     s256 = hq.hq_group_rht_quant_workspace_size(256)
+    assert s256 == 3328                     # the noalloc scratch array is sized to this
     assert s1 >= 4 and s1 % 256 == 0 and s1 <= s32 <= s256
     assert s32 >= 4 * (4 + 3 * 32)          # counter word first, then per-section words
 

@@ -205,6 +205,83 @@ def test_grouped_moe_16384x7168(hq, flags):
     _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
 
 
+def _run_given(hq, x, splits, mask, flags, amax_row=None, amax_col=None, ws=None):
+    """One call with HQ_AMAX_GIVEN: the amax buffers are filled with the given
+    values first and must come back unchanged."""
+    M, K = x.shape
+    S = len(splits)
+    if ws is None:
+        ws = hq.new_workspace(S)
+    out, bufs = _guarded_outputs(hq, M, K, S, flags)
+    if flags & hq.HQ_ROWWISE:
+        out["amax_row"].copy_(torch.from_numpy(np.asarray(amax_row, np.float32)))
+    if flags & hq.HQ_COLWISE:
+        out["amax_col"].copy_(torch.from_numpy(np.asarray(amax_col, np.float32)))
+    hq.group_rht_quant(_bf16_dev(x), splits, mask, flags | hq.HQ_AMAX_GIVEN, ws=ws, out=out)
+    torch.cuda.synchronize()
+    for k, raw in bufs.items():
+        assert torch.all(raw[-GUARD:] == 0xA5), f"guard band of {k} overwritten"
+    assert torch.count_nonzero(ws).item() == 0, "workspace not back in its rest state"
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    if flags & hq.HQ_ROWWISE:
+        assert_bits_equal(got["amax_row"], np.asarray(amax_row, np.float32), "given amax_row changed")
+    if flags & hq.HQ_COLWISE:
+        assert_bits_equal(got["amax_col"], np.asarray(amax_col, np.float32), "given amax_col changed")
+    return got
+
+
+@pytest.mark.parametrize("flags", [3, 1 | 4, 2, 7])
+def test_amax_given_equals_two_pass_result(hq, flags):
+    """Given the amax the two-pass call computes, the single pass reproduces
+    every output of it."""
+    splits = [256, 0, 128, 384]
+    x = _case(491, 256, splits)
+    mask = 0x3C5A
+    first, _ = _run(hq, x, splits, mask, flags)
+    got = _run_given(hq, x, splits, mask, flags, first.get("amax_row"), first.get("amax_col"))
+    for k in first:
+        assert_bits_equal(got[k], first[k], k)
+
+
+def test_amax_given_other_values(hq):
+    """Given values other than the data's amax (above, below: saturation,
+    zero, negative, NaN, and an empty section) against the oracle."""
+    splits = [128, 256, 0, 128, 128]
+    x = _case(493, 384, splits)
+    mask = 0xF00F
+    ref = oracle.group_rht_quant(x, splits, mask, 3)
+    ar = ref["amax_row"] * np.float32([2.0, 0.25, 1.0, 1.0, 1.0])
+    ac = ref["amax_col"] * np.float32([0.5, 3.0, 1.0, 1.0, 1.0])
+    ar[2], ac[2] = 3.0, 0.0                        # empty section
+    ar[3], ac[3] = 0.0, -2.0                       # S_enc = 1
+    ar[4], ac[4] = np.nan, np.float32(1e-35)       # S_enc = 1; S_enc near FLT_MAX (no 0.25 fold)
+    got = _run_given(hq, x, splits, mask, 3, ar, ac)
+    want = oracle.group_rht_quant(x, splits, mask, 3 | oracle.AMAX_GIVEN, amax_row=ar, amax_col=ac)
+    pre = {}
+
+    def pre_of(key):
+        if key not in pre:
+            pre.update(oracle.group_rht_quant(x, splits, mask, 3 | oracle.AMAX_GIVEN, want_pre=True,
+                                              amax_row=ar, amax_col=ac))
+        return pre[key]
+
+    for d in ("row", "col"):
+        assert_bits_equal(got[f"sdec_{d}"], want[f"sdec_{d}"], f"sdec_{d}")
+        assert_bits_equal(got[f"{d}_sf"], want[f"{d}_sf"], f"{d}_sf")
+        assert_fp4_codes(got[f"{d}_codes"], want[f"{d}_codes"], lambda d=d: pre_of(f"{d}_pre"), f"{d} codes")
+
+
+@pytest.mark.slow
+def test_amax_given_grouped_moe_16384x7168(hq):
+    seed = S.SEEDS["grouped_moe"]
+    x = S.normal_bf16(seed, (16384, 7168))
+    splits = S.moe_splits(seed)
+    mask = S.sign_mask16(seed)
+    want = oracle.group_rht_quant(x, splits, mask, 3)
+    got = _run_given(hq, x, splits, mask, 3, want["amax_row"], want["amax_col"])
+    _check(got, want, x, splits, mask, 3)
+
+
 def test_bounded_wait_reports_timeout_and_recovers(hq):
     """A workspace outside its rest state makes the cast tile's wait run out:
     with the tile counter starting at 1, item 0 (the section's only amax tile)
