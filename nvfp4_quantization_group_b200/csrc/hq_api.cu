@@ -189,8 +189,9 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     };
     cudaStream_t st = (cudaStream_t)stream;
     const int max_grid = dev->sms * (dev->nv_blocks_per_sm > 0 ? dev->nv_blocks_per_sm : 1);
-    auto grid_for = [&](uint32_t items) {
-        return (int)(items < (uint32_t)max_grid ? (items > 0 ? items : 1) : (uint32_t)max_grid);
+    auto grid_for = [&](uint32_t items) {  // no more CTAs than claims
+        const uint32_t claims = (items + (uint32_t)nvfp4_tiles_per_claim() - 1) / (uint32_t)nvfp4_tiles_per_claim();
+        return (int)(claims < (uint32_t)max_grid ? (claims > 0 ? claims : 1) : (uint32_t)max_grid);
     };
     auto launch = [&](NvParams& q, uint32_t items) -> hq_status {
         q.seg_start[q.nseg] = items;

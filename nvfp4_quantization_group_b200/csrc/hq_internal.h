@@ -130,10 +130,14 @@ constexpr int NV_CONSUMER_WARPS = HQ_NV_CONSUMER_WARPS;  // compute warps of a C
 constexpr int NV_THREADS = 32 * (NV_CONSUMER_WARPS + 1);  // + the producer warp
 constexpr int NV_STAGES = HQ_NV_STAGES;                  // shared-memory tile buffers per CTA
 constexpr int NV_CTAS_PER_SM = HQ_NV_CTAS_PER_SM;        // resident CTAs the kernel is built for
+#ifndef HQ_NV_CLAIM
+#define HQ_NV_CLAIM 2
+#endif
+constexpr int NV_CLAIM = HQ_NV_CLAIM;                    // consecutive tiles per scheduler claim
 constexpr int NV_MAX_SEG = 2 * HQ_MAX_SECTIONS;
 constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abort
 
-// Workspace words (uint32): [0] tile counter, [1] CTAs finished, [2] sticky
+// Workspace words (uint32): [0] claim counter (claims of NV_CLAIM tiles), [1] CTAs finished, [2] sticky
 // error word (cleared by hq_get_error), [3] abort flag of the running call,
 // then amax_row bits [S], amax_col bits [S], amax-pass tiles finished per
 // section [S].  All but [2] are zero between calls.
@@ -159,6 +163,7 @@ struct NvParams {
 
 int nvfp4_blocks_per_sm();
 int nvfp4_tiles_in_flight_per_cta();  // buffers + the claims in flight
+int nvfp4_tiles_per_claim();
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st);
 
 }  // namespace hq

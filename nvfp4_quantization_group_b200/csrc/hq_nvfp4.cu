@@ -9,12 +9,13 @@
 // buffers (128 x 128 BF16 each).
 //
 //  * The producer claims 128x128 tiles from the workspace's tile counter (two
-//    claims in flight) and writes a small header per buffer.  Before the
-//    first cast tile of a section it waits (bounded) until the section's amax
-//    is complete and fills the buffer's encode tables.  The tile itself comes
-//    in with two TMA loads (the copy engine signals the bytes on the buffer's
-//    "full" mbarrier): no load/store-unit traffic competes with the compute
-//    warps' shared-memory reads.
+//    claims in flight).  As soon as a buffer is free it starts the tile's two
+//    TMA loads (the copy engine signals the bytes on the buffer's "full"
+//    mbarrier: no load/store-unit traffic competes with the compute warps'
+//    shared-memory reads), then, while the copy runs, writes the buffer's
+//    header and, before the first cast tile of a section, waits (bounded)
+//    until the section's amax is complete and fills the buffer's encode
+//    tables.
 //  * Compute warps wait on "full", work on the tile, and release the buffer
 //    on its "empty" mbarrier.  No CTA-wide barrier in the main loop.
 //
@@ -52,6 +53,7 @@ constexpr uint32_t SPIN_LIMIT = 1u << 20;  // section polls of >= 64 ns + a load
 constexpr uint32_t MBAR_LIMIT = 1u << 22;  // barrier sleeps of <= 1 us: far above the section wait
 constexpr int NCW = NV_CONSUMER_WARPS;
 constexpr int NST = NV_STAGES;
+constexpr int CLAIM = NV_CLAIM;  // consecutive tiles per claim
 constexpr int TILE_BYTES = NV_TILE * NV_TILE * 2;
 
 // header flags; H_SLOW_R / H_SLOW_C: the numerator of the per-block encode
@@ -389,21 +391,23 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
     uint32_t* const abort_flag = p.ws + 3;
     const uint32_t total = p.total_items;
     ProducerState ps;
-    // Lane 0 keeps three claims in flight in ca, cb, cc: fill k takes its tile
-    // from one register, refills it with a new claim (read three fills
-    // later) and looks at the next fill's tile, claimed two fills earlier, to
-    // prefetch its section's amax tile count.
-    uint32_t ca = 0, cb = 0, cc = 0;
+    // A claim is CLAIM consecutive tiles (the counter counts claims): one
+    // atomic per CLAIM fills, and consecutive tiles nearly always share their
+    // section, so the section state is looked up less often.  Lane 0 keeps two
+    // claims in flight in ca, cb: the tiles of ca are filled while its
+    // register is refilled with a new claim (read two claims later), and cb,
+    // claimed one claim earlier, gives the tile after the last one (to
+    // prefetch its section's amax tile count).  (More claims in flight
+    // measured slower: tiles are reserved longer before they are worked on,
+    // so sections complete later and the tail is longer.)
+    uint32_t ca = 0, cb = 0;
     if (lane == 0) {
         ca = atomicAdd(counter, 1u);
         cb = atomicAdd(counter, 1u);
-        cc = atomicAdd(counter, 1u);
     }
     uint32_t k = 0;
-    // One buffer fill; false when the producer is done.
-    auto fill = [&](uint32_t& claim, const uint32_t& next) -> bool {
-        const int st = (int)(k % NST);
-        StageHdr& h = sh.hdr[st];
+    // Waits (bounded) until the buffer of fill k is free; false on timeout.
+    auto wait_free = [&](int st) -> bool {
         if (k >= NST && !mbar_wait_bounded(&sh.empty[st], ((k / NST) - 1u) & 1u, MBAR_LIMIT)) {
             if (lane == 0) {
                 atomicOr(err, (uint32_t)HQ_ERR_TIMEOUT);
@@ -411,15 +415,24 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
             }
             return false;  // the compute warps' own bounded waits end them
         }
-        const uint32_t tile = __shfl_sync(0xFFFFFFFFu, claim, 0);
+        return true;
+    };
+    // One buffer fill with `tile` (< total).  The following fill's tile is
+    // `next`, or (last tile of a claim) the first tile of claim cb.
+    auto fill = [&](uint32_t tile, uint32_t next, bool next_from_cb) -> bool {
+        const int st = (int)(k % NST);
+        StageHdr& h = sh.hdr[st];
+        if (!wait_free(st)) return false;
         ++k;
-        if (tile >= total) {  // end of work: an empty header for the compute warps
-            if (lane == 0) h.flags = 0u;
-            mbar_arrive(&sh.full[st]);
-            return false;
-        }
-        if (lane == 0) claim = atomicAdd(counter, 1u);
         const TileInfo t = k == 1u ? decode(p, sh, tile, ps.seg) : ps.nt;
+        if (lane == 0) {
+            // the data first: the header work below overlaps the copy
+            const uint32_t dst = tiles_u32 + (uint32_t)st * TILE_BYTES;
+            const int c1 = (int)(t.row0 / 16);
+            mbar_expect_tx(&sh.full[st], (uint32_t)TILE_BYTES);
+            tma_load_3d(dst, &p.tmap, t.col0, c1, 0, &sh.full[st]);
+            tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, t.col0 + 64, c1, 0, &sh.full[st]);
+        }
         const uint32_t fl = nv_prepare(p, h, t, lane, ps);
         if ((fl & H_CAST) && !(fl & H_GAVE_UP) && sh.enc_section[st] != t.s) {
             // this buffer's encode tables for the section (each lane writes and
@@ -432,16 +445,9 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
             }
             sh.enc_section[st] = t.s;
         }
-        if (lane == 0 && !(fl & H_GAVE_UP)) {
-            const uint32_t dst = tiles_u32 + (uint32_t)st * TILE_BYTES;
-            const int c1 = (int)(t.row0 / 16);
-            mbar_expect_tx(&sh.full[st], (uint32_t)TILE_BYTES);
-            tma_load_3d(dst, &p.tmap, t.col0, c1, 0, &sh.full[st]);
-            tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, t.col0 + 64, c1, 0, &sh.full[st]);
-        }
         mbar_arrive(&sh.full[st]);  // every lane: releases the header writes
-        // ---- prefetch the amax tile count of the next fill's section
-        const uint32_t nt = __shfl_sync(0xFFFFFFFFu, next, 0);
+        // ---- decode the next fill's tile; prefetch its section's amax tile count
+        const uint32_t nt = next_from_cb ? __shfl_sync(0xFFFFFFFFu, cb, 0) * (uint32_t)CLAIM : next;
         if (nt < total) {
             ps.nt = decode(p, sh, nt, ps.seg);
             if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s &&
@@ -452,7 +458,29 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
         }
         return true;
     };
-    while (fill(ca, cb) && fill(cb, cc) && fill(cc, ca)) {
+    for (;;) {
+        const uint32_t first = __shfl_sync(0xFFFFFFFFu, ca, 0) * (uint32_t)CLAIM;
+        if (first >= total) {
+            // end of work: an empty header for the compute warps
+            const int st = (int)(k % NST);
+            if (wait_free(st)) {
+                if (lane == 0) sh.hdr[st].flags = 0u;
+                mbar_arrive(&sh.full[st]);
+                ++k;
+            }
+            break;
+        }
+        if (lane == 0) ca = atomicAdd(counter, 1u);  // read two claims later
+        bool ok = true;
+#pragma unroll 1
+        for (uint32_t j = 0; j < (uint32_t)CLAIM && ok && first + j < total; ++j) {
+            const bool last = j + 1 == (uint32_t)CLAIM || first + j + 1 >= total;
+            ok = fill(first + j, first + j + 1, last);
+        }
+        if (!ok) break;
+        const uint32_t c = ca;  // lane 0: the claim after cb
+        ca = cb;
+        cb = c;
     }
     return k;
 }
@@ -808,10 +836,11 @@ int nvfp4_blocks_per_sm() {
 }
 
 // Tiles per CTA the fused schedule puts between a section's amax and cast
-// segments: the buffers and a claim, enough for the amax tiles to be done
-// and small enough for the rows to stay in L2 (a longer lag is about 1% faster
-// here but reads a third of the input from DRAM twice).
-int nvfp4_tiles_in_flight_per_cta() { return NST + 1; }
+// segments: the buffers and the claims in flight, enough for the amax tiles
+// to be done and small enough for the rows to stay in L2.
+int nvfp4_tiles_in_flight_per_cta() { return NST + 2; }
+
+int nvfp4_tiles_per_claim() { return CLAIM; }
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
     if (p.flags & HQ_ROW_RHT)

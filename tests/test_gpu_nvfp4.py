@@ -283,18 +283,19 @@ def test_amax_given_grouped_moe_16384x7168(hq):
 
 
 def test_bounded_wait_reports_timeout_and_recovers(hq):
-    """A workspace outside its rest state makes the cast tile's wait run out:
-    with the tile counter starting at 1, item 0 (the section's only amax tile)
-    is never claimed, so its cast tile (item 1) waits for an amax that never
-    comes.  The call ends by itself after the bounded spin, hq_get_error
-    reports HQ_ERR_TIMEOUT, the workspace is back at rest and the next call is
-    correct."""
+    """A workspace outside its rest state makes the cast tiles' wait run out:
+    one section of 4 column tiles is 4 amax tiles (items 0..3) then 4 cast
+    tiles; with the claim counter starting at 1, the first claim (item 0, or
+    items 0 and 1 with two tiles per claim) is never made, so the section's
+    amax never completes and its cast tiles wait for it.  The call ends by
+    itself after the bounded spin, hq_get_error reports HQ_ERR_TIMEOUT, the
+    workspace is back at rest and the next call is correct."""
     splits = [128]
-    x = _case(461, 128, splits)
+    x = _case(461, 512, splits)
     ws = hq.new_workspace(1)
     words = ws.view(torch.int32)
-    words[0] = 1                     # tile counter
-    out = hq.group_outputs(128, 128, 1)
+    words[0] = 1                     # claim counter
+    out = hq.group_outputs(128, 512, 1)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
