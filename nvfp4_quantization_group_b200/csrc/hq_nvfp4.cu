@@ -74,12 +74,18 @@ struct alignas(16) StageHdr {  // 48 bytes, moved as three 16-byte words
     float senc_r;      // section encode scale, rowwise (cast tiles)
     float senc_c;      // columnwise
     float senc_cq;     // numerator of the columnwise block encode factor: senc_c, times 0.25 when H_FOLD
+    int32_t tab;       // encode-table slot of the section (cast tiles)
 };
 
 struct NvShared {
     float2 vr[128];  // per E4M3 code: {value, -RN(1 / value)}; {0, -0} for codes 0 and 127
-    float enc[NST][2][128];  // per buffer: S_enc / value(sf) for every code, rowwise and columnwise
-    int32_t enc_section[NST];  // section the buffer's tables hold (producer only)
+    // Encode tables S_enc / value(sf) for every code, rowwise and columnwise,
+    // in NST slots taken in turn at each change of section along the
+    // producer's cast fills.  A slot is rewritten at the NST-th section change
+    // after its own, NST or more fills after the last fill that used it, and
+    // after the producer waited for that fill's buffer to be released.
+    float enc[NST][2][128];
+    int32_t tab_section[NST];  // section a slot holds (producer only)
     StageHdr hdr[NST];
     uint32_t acc_row[NST], acc_col[NST], acc_cnt[NST];  // amax tiles: CTA partial maxima
     uint32_t seg_start[NV_MAX_SEG + 1];  // copies of the schedule (parameter space is slow
@@ -230,6 +236,24 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
     return t;
 }
 
+// decode() of tile = (the tile `prev` describes) + 1, with the cursor where
+// decode() left it for prev: inside the same segment the next row tile, or
+// the first row tile of the next column tile.
+__device__ __forceinline__ TileInfo decode_successor(const NvParams& p, const NvShared& sh, const TileInfo& prev,
+                                                     uint32_t tile, int& seg) {
+    if (seg + 1 < p.nseg && sh.seg_start[seg + 1] <= tile) return decode(p, sh, tile, seg);
+    TileInfo t = prev;
+    if (t.row_in_sec0 + NV_TILE < t.ms) {
+        t.row_in_sec0 += NV_TILE;
+        t.row0 += NV_TILE;
+    } else {
+        t.row_in_sec0 = 0;
+        t.row0 = t.r0s;
+        t.col0 += NV_TILE;
+    }
+    return t;
+}
+
 }  // namespace
 
 namespace {
@@ -280,8 +304,10 @@ struct ProducerState {
     uint32_t r_fl = 0;          // its header flags (H_FOLD, H_SLOW_*, H_GAVE_UP)
     float r_sr = 1.0f, r_srq = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
     uint32_t gave_up = 0;       // sticky once a section wait gave up
-    int pf_s = -1;              // section of the prefetched tile count (lane 0)
+    int pf_s = -1;              // section of the prefetched tile count / given amax (lane 0)
     uint32_t pf = 0;
+    float pf_ar = 0.0f, pf_ac = 0.0f;
+    int tab = 0, tab_s = -1;    // encode-table slot in use and its section
     TileInfo nt;                // the next fill's tile, decoded one fill ahead
 };
 
@@ -304,8 +330,9 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
                 uint64_t rec = 0u;
                 uint32_t g = ps.gave_up;
                 if (p.flags & HQ_AMAX_GIVEN) {
-                    rec = make_record((p.flags & HQ_ROWWISE) ? p.amax_row[t.s] : 0.0f,
-                                      (p.flags & HQ_COLWISE) ? p.amax_col[t.s] : 0.0f);
+                    const bool pre = ps.pf_s == t.s;  // prefetched with the tile
+                    rec = make_record((p.flags & HQ_ROWWISE) ? (pre ? ps.pf_ar : p.amax_row[t.s]) : 0.0f,
+                                      (p.flags & HQ_COLWISE) ? (pre ? ps.pf_ac : p.amax_col[t.s]) : 0.0f);
                 } else if (!g) {
                     const uint32_t* const done = p.ws + NV_WS_HEADER + 2 * p.S + t.s;
                     const uint32_t target = (uint32_t)(t.ms / NV_TILE) * (uint32_t)p.col_tiles;
@@ -374,6 +401,7 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
         v.senc_r = ps.r_sr;
         v.senc_c = ps.r_sc;
         v.senc_cq = ps.r_scq;
+        v.tab = ps.tab;
         const uint4* src = reinterpret_cast<const uint4*>(&v);
         uint4* dst = reinterpret_cast<uint4*>(&h);
         dst[0] = src[0];
@@ -433,26 +461,32 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
             tma_load_3d(dst, &p.tmap, t.col0, c1, 0, &sh.full[st]);
             tma_load_3d(dst + TILE_BYTES / 2, &p.tmap, t.col0 + 64, c1, 0, &sh.full[st]);
         }
+        if (t.phase == 1 && t.s != ps.tab_s) {
+            ps.tab = ps.tab + 1 == NST ? 0 : ps.tab + 1;  // a new section: the next table slot
+            ps.tab_s = t.s;
+        }
         const uint32_t fl = nv_prepare(p, h, t, lane, ps);
-        if ((fl & H_CAST) && !(fl & H_GAVE_UP) && sh.enc_section[st] != t.s) {
-            // this buffer's encode tables for the section (each lane writes and
-            // later reads only the value it wrote itself into enc_section)
+        if ((fl & H_CAST) && !(fl & H_GAVE_UP) && sh.tab_section[ps.tab] != t.s) {
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const uint32_t code = (uint32_t)lane + 32u * m;
-                sh.enc[st][0][code] = block_enc(sh, code, ps.r_srq, fl & H_SLOW_R);
-                sh.enc[st][1][code] = block_enc(sh, code, ps.r_scq, fl & H_SLOW_C);
+                sh.enc[ps.tab][0][code] = block_enc(sh, code, ps.r_srq, fl & H_SLOW_R);
+                sh.enc[ps.tab][1][code] = block_enc(sh, code, ps.r_scq, fl & H_SLOW_C);
             }
-            sh.enc_section[st] = t.s;
+            sh.tab_section[ps.tab] = t.s;  // (each lane reads back only its own write)
         }
         mbar_arrive(&sh.full[st]);  // every lane: releases the header writes
         // ---- decode the next fill's tile; prefetch its section's amax tile count
         const uint32_t nt = next_from_cb ? __shfl_sync(0xFFFFFFFFu, cb, 0) * (uint32_t)CLAIM : next;
         if (nt < total) {
-            ps.nt = decode(p, sh, nt, ps.seg);
-            if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s &&
-                !(p.flags & HQ_AMAX_GIVEN)) {
-                ps.pf = ld_relaxed_u32(p.ws + NV_WS_HEADER + 2 * p.S + ps.nt.s);
+            ps.nt = next_from_cb ? decode(p, sh, nt, ps.seg) : decode_successor(p, sh, t, nt, ps.seg);
+            if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s) {
+                if (p.flags & HQ_AMAX_GIVEN) {
+                    ps.pf_ar = (p.flags & HQ_ROWWISE) ? p.amax_row[ps.nt.s] : 0.0f;
+                    ps.pf_ac = (p.flags & HQ_COLWISE) ? p.amax_col[ps.nt.s] : 0.0f;
+                } else {
+                    ps.pf = ld_relaxed_u32(p.ws + NV_WS_HEADER + 2 * p.S + ps.nt.s);
+                }
                 ps.pf_s = ps.nt.s;
             }
         }
@@ -648,7 +682,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 for (int i = 0; i < 16; ++i) unpack2(v[i], r0[i], r1[i]);
                 const uint32_t sf0 = block_sf(__fmul_rn(absmax16(r0), 0.25f), h.senc_r);
                 const uint32_t sf1 = block_sf(__fmul_rn(absmax16(r1), 0.25f), h.senc_r);
-                const f2 e2 = pack2(sh.enc[st][0][sf0], sh.enc[st][0][sf1]);
+                const f2 e2 = pack2(sh.enc[h.tab][0][sf0], sh.enc[h.tab][0][sf1]);
                 if (!(h.flags & H_FOLD_R)) {
                     const f2 quarter = pack2(0.25f, 0.25f);
 #pragma unroll
@@ -676,7 +710,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     const uint32_t m = hmax_abs(hmax_abs(hmax_abs(wd[0], wd[1]), hmax_abs(wd[2], wd[3])),
                                                 hmax_abs(hmax_abs(wd[4], wd[5]), hmax_abs(wd[6], wd[7])));
                     const uint32_t sf = block_sf(__uint_as_float(halves_max_bits(m)), h.senc_r);
-                    const float enc = sh.enc[st][0][sf];
+                    const float enc = sh.enc[h.tab][0][sf];
                     const f2 e2 = pack2(enc, enc);
                     float q[16];
 #pragma unroll
@@ -705,7 +739,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 const float a0 = absmax16(c0), a1 = absmax16(c1);
                 const uint32_t sf0 = block_sf(__fmul_rn(a0, 0.25f), h.senc_c);
                 const uint32_t sf1 = block_sf(__fmul_rn(a1, 0.25f), h.senc_c);
-                const f2 e2 = pack2(sh.enc[st][1][sf0], sh.enc[st][1][sf1]);
+                const f2 e2 = pack2(sh.enc[h.tab][1][sf0], sh.enc[h.tab][1][sf1]);
                 if (!(h.flags & H_FOLD)) {
                     const f2 quarter = pack2(0.25f, 0.25f);
 #pragma unroll
@@ -759,7 +793,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
             sh.acc_row[st] = 0u;
             sh.acc_col[st] = 0u;
             sh.acc_cnt[st] = 0u;
-            sh.enc_section[st] = -1;
+            sh.tab_section[st] = -1;
         }
         fence_mbar_init();
     }
