@@ -89,7 +89,8 @@ struct NvShared {
     StageHdr hdr[NST];
     uint32_t acc_row[NST], acc_col[NST], acc_cnt[NST];  // amax tiles: CTA partial maxima
     uint32_t seg_start[NV_MAX_SEG + 1];  // copies of the schedule (parameter space is slow
-    uint16_t seg_info[NV_MAX_SEG];       //   to index dynamically)
+    uint32_t seg_off[NV_MAX_SEG];        //   to index dynamically)
+    uint16_t seg_info[NV_MAX_SEG];
     int32_t sec_row0[HQ_MAX_SECTIONS + 1];
     uint32_t sec_magic[HQ_MAX_SECTIONS];  // floor((2^32 - 1) / row tiles of the section)
     uint64_t full[NST], empty[NST];
@@ -219,7 +220,7 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
     TileInfo t;
     t.s = (int)(info & 0x7FFFu);
     t.phase = (int)(info >> 15);
-    const uint32_t local = tile - sh.seg_start[seg];
+    const uint32_t local = tile - sh.seg_start[seg] + sh.seg_off[seg];
     t.r0s = sh.sec_row0[t.s];
     t.ms = sh.sec_row0[t.s + 1] - t.r0s;
     t.trows = t.ms / NV_TILE;
@@ -278,6 +279,11 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* q) {
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(q) : "memory");
     return v;
 }
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* q) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(q) : "memory");
+    return v;
+}
 // with a relaxed load before it that saw the final count: an acquire pattern
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void red_max_u32(uint32_t* q, uint32_t v) {
@@ -304,7 +310,10 @@ struct ProducerState {
     uint32_t r_fl = 0;          // its header flags (H_FOLD, H_SLOW_*, H_GAVE_UP)
     float r_sr = 1.0f, r_srq = 1.0f, r_sc = 1.0f, r_scq = 1.0f;
     uint32_t gave_up = 0;       // sticky once a section wait gave up
-    int pf_s = -1;              // section of the prefetched tile count / given amax (lane 0)
+    // Prefetched one fill ahead for the next tile's section (lane 0): its
+    // amax tile count (an acquire load) and, after it, its maxima (final when
+    // the count is complete), or the caller's amax.
+    int pf_s = -1;
     uint32_t pf = 0;
     float pf_ar = 0.0f, pf_ac = 0.0f;
     int tab = 0, tab_s = -1;    // encode-table slot in use and its section
@@ -337,6 +346,7 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
                     const uint32_t* const done = p.ws + NV_WS_HEADER + 2 * p.S + t.s;
                     const uint32_t target = (uint32_t)(t.ms / NV_TILE) * (uint32_t)p.col_tiles;
                     uint32_t d = ps.pf_s == t.s ? ps.pf : ld_relaxed_u32(done);
+                    const bool pf_final = ps.pf_s == t.s && d >= target;  // the prefetched maxima are final
                     uint32_t spins = 0;
                     while (!g && d < target) {
                         if (*(volatile uint32_t*)abort_flag != 0u) {
@@ -350,7 +360,9 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
                             d = ld_relaxed_u32(done);
                         }
                     }
-                    if (!g) {
+                    if (pf_final) {
+                        rec = make_record(ps.pf_ar, ps.pf_ac);
+                    } else if (!g) {
                         fence_acq_rel_gpu();  // every counted tile's maxima are visible now
                         rec = make_record(__uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + t.s)),
                                           __uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + p.S + t.s)));
@@ -485,7 +497,10 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
                     ps.pf_ar = (p.flags & HQ_ROWWISE) ? p.amax_row[ps.nt.s] : 0.0f;
                     ps.pf_ac = (p.flags & HQ_COLWISE) ? p.amax_col[ps.nt.s] : 0.0f;
                 } else {
-                    ps.pf = ld_relaxed_u32(p.ws + NV_WS_HEADER + 2 * p.S + ps.nt.s);
+                    // the acquire orders the maxima loads after the count
+                    ps.pf = ld_acquire_u32(p.ws + NV_WS_HEADER + 2 * p.S + ps.nt.s);
+                    ps.pf_ar = __uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + ps.nt.s));
+                    ps.pf_ac = __uint_as_float(ld_relaxed_u32(p.ws + NV_WS_HEADER + p.S + ps.nt.s));
                 }
                 ps.pf_s = ps.nt.s;
             }
@@ -798,7 +813,10 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
         fence_mbar_init();
     }
     for (int i = tid; i <= p.nseg; i += NV_THREADS) sh.seg_start[i] = p.seg_start[i];
-    for (int i = tid; i < p.nseg; i += NV_THREADS) sh.seg_info[i] = p.seg_info[i];
+    for (int i = tid; i < p.nseg; i += NV_THREADS) {
+        sh.seg_info[i] = p.seg_info[i];
+        sh.seg_off[i] = p.seg_off[i];
+    }
     for (int i = tid; i <= p.S; i += NV_THREADS) sh.sec_row0[i] = p.sec_row0[i];
     for (int i = tid; i < p.S; i += NV_THREADS) {
         const uint32_t trows = (uint32_t)(p.sec_row0[i + 1] - p.sec_row0[i]) / NV_TILE;
