@@ -198,13 +198,17 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     auto add_seg = [&](NvParams& q, int s, int phase, uint32_t& next) { add_range(q, s, phase, 0, tiles_of(s), next); };
     cudaStream_t st = (cudaStream_t)stream;
     const int max_grid = dev->sms * (dev->nv_blocks_per_sm > 0 ? dev->nv_blocks_per_sm : 1);
+    const uint32_t per_claim = (uint32_t)nvfp4_tiles_per_claim();
     auto grid_for = [&](uint32_t items) {  // no more CTAs than claims
-        const uint32_t claims = (items + (uint32_t)nvfp4_tiles_per_claim() - 1) / (uint32_t)nvfp4_tiles_per_claim();
+        const uint32_t claims = (items + per_claim - 1) / per_claim;
         return (int)(claims < (uint32_t)max_grid ? (claims > 0 ? claims : 1) : (uint32_t)max_grid);
     };
     auto launch = [&](NvParams& q, uint32_t items) -> hq_status {
         q.seg_start[q.nseg] = items;
         q.total_items = items;
+        // multi-tile claims, then single tiles for about two per CTA at the end
+        const uint32_t tail = 2u * (uint32_t)grid_for(items);
+        q.multi_claims = items > tail ? (items - tail) / per_claim : 0u;
         launch_nvfp4(q, grid_for(items), st);
         return launch_status();
     };

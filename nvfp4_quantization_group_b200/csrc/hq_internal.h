@@ -154,6 +154,7 @@ struct NvParams {
     int col_tiles;      // K / 128
     int nseg;           // schedule segments
     uint32_t total_items;
+    uint32_t multi_claims;  // claims of NV_CLAIM tiles; the claims after them take one tile each
     int finalize;       // last launch of the call: publish amax/sdec, reset ws
     int reset_counter;  // reset the tile counter / exit count at the end
     int sec_row0[HQ_MAX_SECTIONS + 1];

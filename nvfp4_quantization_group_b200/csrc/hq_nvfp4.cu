@@ -433,13 +433,18 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
     ProducerState ps;
     // A claim is CLAIM consecutive tiles (the counter counts claims): one
     // atomic per CLAIM fills, and consecutive tiles nearly always share their
-    // section, so the section state is looked up less often.  Lane 0 keeps two
+    // section, so the section state is looked up less often.  The last tiles
+    // (about two per CTA; host's choice) go one per claim, for an even tail.  Lane 0 keeps two
     // claims in flight in ca, cb: the tiles of ca are filled while its
     // register is refilled with a new claim (read two claims later), and cb,
     // claimed one claim earlier, gives the tile after the last one (to
     // prefetch its section's amax tile count).  (More claims in flight
     // measured slower: tiles are reserved longer before they are worked on,
     // so sections complete later and the tail is longer.)
+    // first tile of a claim
+    auto claim_first = [&](uint32_t c) -> uint32_t {
+        return c < p.multi_claims ? c * (uint32_t)CLAIM : c + p.multi_claims * (uint32_t)(CLAIM - 1);
+    };
     uint32_t ca = 0, cb = 0;
     if (lane == 0) {
         ca = atomicAdd(counter, 1u);
@@ -489,7 +494,7 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
         }
         mbar_arrive(&sh.full[st]);  // every lane: releases the header writes
         // ---- decode the next fill's tile; prefetch its section's amax tile count
-        const uint32_t nt = next_from_cb ? __shfl_sync(0xFFFFFFFFu, cb, 0) * (uint32_t)CLAIM : next;
+        const uint32_t nt = next_from_cb ? claim_first(__shfl_sync(0xFFFFFFFFu, cb, 0)) : next;
         if (nt < total) {
             ps.nt = next_from_cb ? decode(p, sh, nt, ps.seg) : decode_successor(p, sh, t, nt, ps.seg);
             if (lane == 0 && ps.nt.phase == 1 && ps.nt.s != ps.ready_s && ps.nt.s != ps.pf_s) {
@@ -508,7 +513,9 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
         return true;
     };
     for (;;) {
-        const uint32_t first = __shfl_sync(0xFFFFFFFFu, ca, 0) * (uint32_t)CLAIM;
+        const uint32_t claim = __shfl_sync(0xFFFFFFFFu, ca, 0);
+        const uint32_t first = claim_first(claim);
+        const uint32_t count = claim < p.multi_claims ? (uint32_t)CLAIM : 1u;
         if (first >= total) {
             // end of work: an empty header for the compute warps
             const int st = (int)(k % NST);
@@ -522,8 +529,8 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
         if (lane == 0) ca = atomicAdd(counter, 1u);  // read two claims later
         bool ok = true;
 #pragma unroll 1
-        for (uint32_t j = 0; j < (uint32_t)CLAIM && ok && first + j < total; ++j) {
-            const bool last = j + 1 == (uint32_t)CLAIM || first + j + 1 >= total;
+        for (uint32_t j = 0; j < count && ok && first + j < total; ++j) {
+            const bool last = j + 1 == count || first + j + 1 >= total;
             ok = fill(first + j, first + j + 1, last);
         }
         if (!ok) break;
