@@ -181,21 +181,12 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     p.sec_row0[S] = row0;
 
     auto tiles_of = [&](int s) { return (uint32_t)(split_rows[s] / NV_TILE) * (uint32_t)p.col_tiles; };
-    // a segment: `len` tiles of section s (phase 0 amax, 1 cast) from tile
-    // `off` of the section's tile order
-    bool seg_overflow = false;  // (cannot happen: the chunk size keeps the table in bounds)
-    auto add_range = [&](NvParams& q, int s, int phase, uint32_t off, uint32_t len, uint32_t& next) {
-        if (q.nseg >= NV_MAX_SEG) {
-            seg_overflow = true;
-            return;
-        }
+    auto add_seg = [&](NvParams& q, int s, int phase, uint32_t& next) {
         q.seg_start[q.nseg] = next;
         q.seg_info[q.nseg] = (uint16_t)(s | (phase << 15));
-        q.seg_off[q.nseg] = off;
         ++q.nseg;
-        next += len;
+        next += tiles_of(s);
     };
-    auto add_seg = [&](NvParams& q, int s, int phase, uint32_t& next) { add_range(q, s, phase, 0, tiles_of(s), next); };
     cudaStream_t st = (cudaStream_t)stream;
     const int max_grid = dev->sms * (dev->nv_blocks_per_sm > 0 ? dev->nv_blocks_per_sm : 1);
     const uint32_t per_claim = (uint32_t)nvfp4_tiles_per_claim();
@@ -223,50 +214,31 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
         return launch(p, next);
     }
     if (!(flags & HQ_TWO_PASS)) {
-        // One launch.  Amax and cast tiles alternate in chunks of about one
-        // tile per CTA, so that every CTA's buffer ring sees a steady mix (on a
-        // long run of amax tiles, which are quicker to work on, the compute
-        // warps outrun the copies).  A section's cast chunks come after all
-        // its amax chunks and `lag` more tiles (the tiles the grid holds in
-        // flight), so its amax is normally complete when its first cast tile
-        // is claimed and its rows are still in L2; every tile depends only on
-        // tiles scheduled before it.
-        uint32_t all = 0, all_a = 0;
-        for (int k = 0; k < nlive; ++k) all_a += tiles_of(live[k]);
-        all = 2 * all_a;
-        const uint32_t grid = (uint32_t)grid_for(all);
-        const uint32_t lag = grid * (uint32_t)nvfp4_tiles_in_flight_per_cta();
-        // chunks per phase: at most one per section plus `room`, within the
-        // segment table (sum of ceil(T_s / chunk) <= nlive + all_a / chunk)
-        const uint32_t room = (uint32_t)(NV_MAX_SEG / 2 - nlive);
-        uint32_t chunk = grid > 64u ? grid : 64u;
-        if (room == 0) chunk = 0xFFFFFFFFu;
-        else if (chunk < (all_a + room - 1) / room) chunk = (all_a + room - 1) / room;
-        struct Pending { int s; uint32_t ready, off; };
-        Pending cq[HQ_MAX_SECTIONS];  // sections whose amax is scheduled, in that order
-        int ch = 0, ct = 0, ka = 0;
-        uint32_t a_off = 0, next = 0;
-        while (ka < nlive || ch < ct) {
-            if (ch < ct && (cq[ch].ready <= next || ka >= nlive)) {
-                const uint32_t T = tiles_of(cq[ch].s);
-                const uint32_t len = T - cq[ch].off < chunk ? T - cq[ch].off : chunk;
-                add_range(p, cq[ch].s, 1, cq[ch].off, len, next);
-                cq[ch].off += len;
-                if (cq[ch].off == T) ++ch;
-            }
-            if (ka < nlive) {
-                const uint32_t T = tiles_of(live[ka]);
-                const uint32_t len = T - a_off < chunk ? T - a_off : chunk;
-                add_range(p, live[ka], 0, a_off, len, next);
-                a_off += len;
-                if (a_off == T) {
-                    cq[ct++] = Pending{live[ka], next + lag, 0u};
-                    ++ka;
-                    a_off = 0;
-                }
+        // One launch.  The cast segment of a section follows its amax segment
+        // once `lag` more tiles have been scheduled (the tiles the grid holds
+        // in flight), so its amax is normally complete when its first tile is
+        // claimed and its rows are still in L2 (the distance between a tile's
+        // two reads is the section's tiles plus the lag; interleaving amax and
+        // cast tiles more finely measured no faster and doubled that distance
+        // for the first tiles, reading a third more from DRAM).  Every tile
+        // depends only on tiles scheduled before it.
+        uint32_t all = 0;
+        for (int k = 0; k < nlive; ++k) all += 2 * tiles_of(live[k]);
+        const uint32_t lag = (uint32_t)grid_for(all) * (uint32_t)nvfp4_tiles_in_flight_per_cta();
+        uint32_t next = 0, a_end[HQ_MAX_SECTIONS];
+        int pend = 0;  // next section whose cast segment is still to be scheduled
+        for (int k = 0; k < nlive; ++k) {
+            add_seg(p, live[k], 0, next);
+            a_end[k] = next;
+            while (pend < k && next - a_end[pend] >= lag) {
+                add_seg(p, live[pend], 1, next);
+                ++pend;
             }
         }
-        if (seg_overflow) return HQ_ERR_SHAPE;
+        while (pend < nlive) {
+            add_seg(p, live[pend], 1, next);
+            ++pend;
+        }
         p.finalize = 1;
         p.reset_counter = 1;
         return launch(p, next);

@@ -160,7 +160,6 @@ struct NvParams {
     int sec_row0[HQ_MAX_SECTIONS + 1];
     uint32_t seg_start[NV_MAX_SEG + 1];
     uint16_t seg_info[NV_MAX_SEG];  // section | (phase << 15); phase 0 amax, 1 cast
-    uint32_t seg_off[NV_MAX_SEG];   // the segment's first tile inside its section's tile order
 };
 
 int nvfp4_blocks_per_sm();

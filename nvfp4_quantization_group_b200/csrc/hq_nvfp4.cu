@@ -89,8 +89,7 @@ struct NvShared {
     StageHdr hdr[NST];
     uint32_t acc_row[NST], acc_col[NST], acc_cnt[NST];  // amax tiles: CTA partial maxima
     uint32_t seg_start[NV_MAX_SEG + 1];  // copies of the schedule (parameter space is slow
-    uint32_t seg_off[NV_MAX_SEG];        //   to index dynamically)
-    uint16_t seg_info[NV_MAX_SEG];
+    uint16_t seg_info[NV_MAX_SEG];       //   to index dynamically)
     int32_t sec_row0[HQ_MAX_SECTIONS + 1];
     uint32_t sec_magic[HQ_MAX_SECTIONS];  // floor((2^32 - 1) / row tiles of the section)
     uint64_t full[NST], empty[NST];
@@ -220,7 +219,7 @@ __device__ __forceinline__ TileInfo decode(const NvParams& p, const NvShared& sh
     TileInfo t;
     t.s = (int)(info & 0x7FFFu);
     t.phase = (int)(info >> 15);
-    const uint32_t local = tile - sh.seg_start[seg] + sh.seg_off[seg];
+    const uint32_t local = tile - sh.seg_start[seg];
     t.r0s = sh.sec_row0[t.s];
     t.ms = sh.sec_row0[t.s + 1] - t.r0s;
     t.trows = t.ms / NV_TILE;
@@ -820,10 +819,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
         fence_mbar_init();
     }
     for (int i = tid; i <= p.nseg; i += NV_THREADS) sh.seg_start[i] = p.seg_start[i];
-    for (int i = tid; i < p.nseg; i += NV_THREADS) {
-        sh.seg_info[i] = p.seg_info[i];
-        sh.seg_off[i] = p.seg_off[i];
-    }
+    for (int i = tid; i < p.nseg; i += NV_THREADS) sh.seg_info[i] = p.seg_info[i];
     for (int i = tid; i <= p.S; i += NV_THREADS) sh.sec_row0[i] = p.sec_row0[i];
     for (int i = tid; i < p.S; i += NV_THREADS) {
         const uint32_t trows = (uint32_t)(p.sec_row0[i + 1] - p.sec_row0[i]) / NV_TILE;
