@@ -62,6 +62,9 @@ def lib() -> ctypes.CDLL:
             L.hqo_cat_rotate_fp8.argtypes = [P, i64, ctypes.c_int, P, i64, ctypes.c_int, i64,
                                              ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, i64, P, P]
             L.hqo_cat_rotate_fp8.restype = ctypes.c_int
+            L.hqo_cat_rotate_nvfp4.argtypes = [P, i64, ctypes.c_int, P, i64, ctypes.c_int, i64,
+                                               ctypes.c_int, ctypes.c_int, P, P, P, ctypes.c_int, i64, P, P]
+            L.hqo_cat_rotate_nvfp4.restype = ctypes.c_int
             L.hqo_swiglu_fp8_k128.argtypes = [ctypes.c_int, P, i64, i64, P, P, P, P]
             L.hqo_swiglu_fp8_k128.restype = ctypes.c_int
             L.hqo_group_rht_quant.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_uint16, ctypes.c_uint,
@@ -152,6 +155,43 @@ def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=N
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return (out, scales, pre, amax) if want_amax else (out, scales, pre)
+
+
+def cat_rotate_nvfp4(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=None,
+                     scale_layout=ROWMAJOR, scale_ld=None, want_pre=False, want_amax=False):
+    """Concat (a | b) per group, optional 128-point Hadamard, NVFP4 per
+    128-vector (8 blocks of 16, E4M3 block scales, per-vector decode scale).
+
+    Returns a dict: codes [M, G*64] uint8, block_sf [M, G*8] uint8, sdec
+    (scales' layout), and amax / pre when asked.
+    """
+    a = np.ascontiguousarray(a, dtype=np.uint16)
+    a_w = int(a.shape[-1])
+    a_rs = a_row_stride if a_row_stride is not None else G * a_w
+    if b is not None:
+        b = np.ascontiguousarray(b, dtype=np.uint16)
+        b_w = int(b.shape[-1])
+        b_rs = b_row_stride if b_row_stride is not None else G * b_w
+    else:
+        b_w, b_rs = 0, 0
+    r = {"codes": np.empty((M, G * 64), dtype=np.uint8), "block_sf": np.empty((M, G * 8), dtype=np.uint8)}
+    if scale_layout == ROWMAJOR:
+        r["sdec"] = np.empty((M, G), dtype=np.float32)
+        ld = G
+    else:
+        ld = scale_ld if scale_ld is not None else M
+        r["sdec"] = np.zeros((G, ld), dtype=np.float32)
+    if want_amax:
+        r["amax"] = np.zeros_like(r["sdec"])
+    if want_pre:
+        r["pre"] = np.empty((M, G * 128), dtype=np.float32)
+    g = r.get
+    rc = lib().hqo_cat_rotate_nvfp4(_ptr(a), a_rs, a_w, _ptr(b), b_rs, b_w, M, G, hadamard_n,
+                                    _ptr(r["codes"]), _ptr(r["block_sf"]), _ptr(r["sdec"]), scale_layout, ld,
+                                    _ptr(g("amax")), _ptr(g("pre")))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return r
 
 
 NONE_BF16, NONE_F32, SWIGLU_F32 = 0, 1, 2

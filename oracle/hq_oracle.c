@@ -535,3 +535,59 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------ FP4 DSA */
+/*
+ * The DSA indexer prep with an NVFP4 output instead of FP8 ([DSA]: the FP4
+ * path, fused_cat_fp4, lacks the rotation; restoring it is the follow-up the
+ * page names).  The pages give no FP4 format; reading: the vector (t, g) is
+ * concatenated and rotated exactly as in hqo_cat_rotate_fp8, then quantized
+ * with the two-level NVFP4 scheme of hqo_group_rht_quant, the 128-vector
+ * taking the place of a section:
+ *   A = max |v| over the 128 values, S_enc = global_encode_scale(A),
+ *   eight blocks of 16 consecutive values: E4M3 block scale and E2M1 codes
+ *   (nvfp4_block), the vector's decode scale 1/S_enc stored like the FP8
+ *   scales (row major [M, G] or transposed [G, scale_ld]).
+ * codes: [M, G*64] bytes (vector (t, g) at (t*G + g)*64, element 2k in the
+ * low nibble); block_sf: [M, G*8] E4M3 codes; amax_opt: A per vector in the
+ * scales' layout; pre: the value rounded to E2M1 per element, [M, G*128].
+ * Returns 0, or -1 for arguments this reference does not accept.
+ */
+int hqo_cat_rotate_nvfp4(const uint16_t *a, int64_t a_row_stride, int a_width,
+                         const uint16_t *b, int64_t b_row_stride, int b_width,
+                         int64_t M, int G, int hadamard_n,
+                         uint8_t *codes, uint8_t *block_sf, float *sdec, int scale_layout, int64_t scale_ld,
+                         float *amax_opt, float *pre)
+{
+    if (a_width < 0 || b_width < 0 || a_width + b_width != 128 || (b_width > 0 && !b))
+        return -1;
+    if (hadamard_n != 0 && hadamard_n != 128)
+        return -1;
+    const float c = c128();
+    float v[128];
+    for (int64_t t = 0; t < M; ++t)
+        for (int g = 0; g < G; ++g) {
+            for (int j = 0; j < a_width; ++j)
+                v[j] = bf16_value(a[t * a_row_stride + (int64_t)g * a_width + j]);
+            for (int j = 0; j < b_width; ++j)
+                v[a_width + j] = bf16_value(b[t * b_row_stride + (int64_t)g * b_width + j]);
+            if (hadamard_n == 128) {
+                hqo_fwht(v, 128);
+                for (int j = 0; j < 128; ++j)
+                    v[j] = v[j] * c;
+            }
+            float A = 0.0f;
+            for (int j = 0; j < 128; ++j)
+                A = fmaxf(A, fabsf(v[j]));
+            const float S_enc = global_encode_scale(A);
+            const int64_t vec = t * G + g;
+            for (int blk = 0; blk < 8; ++blk)
+                nvfp4_block(v + 16 * blk, S_enc, codes + vec * 64 + 8 * blk, block_sf + vec * 8 + blk,
+                            pre ? pre + vec * 128 + 16 * blk : 0);
+            const int64_t si = scale_layout == 0 ? vec : (int64_t)g * scale_ld + t;
+            sdec[si] = 1.0f / S_enc;
+            if (amax_opt)
+                amax_opt[si] = A;
+        }
+    return 0;
+}

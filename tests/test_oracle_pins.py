@@ -588,6 +588,76 @@ def test_nvfp4_amax_given_single_pass():
         np.testing.assert_array_equal(w[k], z[k], err_msg=k)
 
 
+def test_fp4_dsa_without_rotation_follows_the_nvfp4_rule():
+    """cat -> NVFP4 per 128-vector (no rotation): vector amax, decode scale,
+    block scales and codes follow the closed-form two-level rule."""
+    M, G = 5, 3
+    pe = S.normal_bf16(311, (M, G, 64))
+    nope = S.with_outliers_bf16(S.normal_bf16(312, (M, G, 64)), 313, p=0.02)
+    pe[2, 1] = 0
+    nope[2, 1] = 0                                    # an all-zero vector
+    r = oracle.cat_rotate_nvfp4(pe, nope, M, G, 0, want_pre=True, want_amax=True)
+    v = np.concatenate([S.bf16_bits_to_f32(pe), S.bf16_bits_to_f32(nope)], axis=-1)   # [M, G, 128]
+    A = np.max(np.abs(v), axis=-1)
+    np.testing.assert_array_equal(r["amax"], A)
+    nib = _unpack(r["codes"]).reshape(M, G, 8, 16)
+    sf = r["block_sf"].reshape(M, G, 8)
+    pre = r["pre"].reshape(M, G, 8, 16)
+    for t in range(M):
+        for g in range(G):
+            if A[t, g] == 0:
+                assert r["sdec"][t, g] == 1 and np.all(sf[t, g] == 0) and np.all((nib[t, g] & 7) == 0)
+                continue
+            S_enc = np.float32(2688) / A[t, g]
+            assert r["sdec"][t, g] == np.float32(1) / S_enc
+            blocks = v[t, g].reshape(8, 16)
+            ab = np.max(np.abs(blocks), axis=-1)
+            for k in range(8):
+                want = nearest_code(frac(ab[k]) / 6 * frac(S_enc), E4C, E4V, 0x80, False)
+                if sf[t, g, k] != want:
+                    assert near_midpoint(frac(ab[k]) / 6 * frac(S_enc), E4V)
+            assert sf[t, g, int(np.argmax(ab))] == 0x7E        # the block holding the amax
+            sff = _e4m3_vals(sf[t, g]).astype(np.float32)
+            enc = np.where(sff == 0, 0, S_enc / sff).astype(np.float32)
+            np.testing.assert_array_equal(pre[t, g], (blocks * enc[:, None]).astype(np.float32))
+            for k in range(8):
+                for i in range(16):
+                    want = nearest_code(frac(pre[t, g, k, i]), E2C, E2V, 0x8, is_negative(pre[t, g, k, i]))
+                    if nib[t, g, k, i] != want:
+                        assert near_midpoint(frac(pre[t, g, k, i]), E2V)
+
+
+def test_fp4_dsa_rotation_and_layouts():
+    """With the rotation: the pre-rounding values are the dense FP64 rotation
+    times the block encode factors, the dequantized vector rotates back to
+    x within the NVFP4 bound, the amax equals the FP8 path's, and the
+    transposed layout puts vector (t, g) at sdec[g, t]."""
+    M, G = 6, 4
+    pe = S.normal_bf16(321, (M, G, 64))
+    nope = S.normal_bf16(322, (M, G, 64))
+    r = oracle.cat_rotate_nvfp4(pe, nope, M, G, 128, want_pre=True, want_amax=True)
+    x = np.concatenate([S.bf16_bits_to_f32(pe), S.bf16_bits_to_f32(nope)], axis=-1).astype(np.float64)
+    H = scipy.linalg.hadamard(128).astype(np.float64) / math.sqrt(128)
+    y = x @ H.T                                                             # [M, G, 128]
+    assert np.max(np.abs(r["amax"] - np.max(np.abs(y), axis=-1)) / r["amax"]) <= 2e-6
+    _, _, _, am8 = oracle.cat_rotate_fp8(pe, nope, M, G, 128, want_amax=True)
+    np.testing.assert_array_equal(r["amax"], am8)
+    sff = _e4m3_vals(r["block_sf"]).reshape(M, G, 8)
+    S_enc = (1.0 / r["sdec"].astype(np.float64))[..., None]
+    enc = np.where(sff == 0, 0, S_enc / sff)
+    v = r["pre"].reshape(M, G, 8, 16) / np.where(enc == 0, 1, enc)[..., None]
+    assert np.max(np.abs(v.reshape(M, G, 128) - y)) <= 1e-5 * np.max(np.linalg.norm(x, axis=-1))
+    deq = _e2m1_vals(_unpack(r["codes"])).reshape(M, G, 8, 16) * (sff / S_enc)[..., None]
+    back = deq.reshape(M, G, 128) @ H                                       # H orthonormal, symmetric
+    ab = np.max(np.abs(y.reshape(M, G, 8, 16)), axis=-1)
+    err = np.linalg.norm(back - x, axis=-1)
+    assert np.all(err <= np.linalg.norm(ab / 6 * 1.07, axis=-1) * 4 + 1e-30)
+    rt = oracle.cat_rotate_nvfp4(pe, nope, M, G, 128, scale_layout=oracle.TRANSPOSED, scale_ld=8)
+    np.testing.assert_array_equal(rt["sdec"][:, :M], r["sdec"].T)
+    assert np.all(rt["sdec"][:, M:] == 0)
+    np.testing.assert_array_equal(rt["codes"], r["codes"])
+
+
 def test_nvfp4_zero_section_and_tiny_values():
     x = np.zeros((256, 128), dtype=np.uint16)
     x[128:] = S.normal_bf16(97, (128, 128))
