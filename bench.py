@@ -55,7 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="grouped_moe",
                     choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4",
-                             "dsa_indexer", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
+                             "dsa_indexer", "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
     ap.add_argument("--no-extras", action="store_true", help="time only the headline workload")
     ap.add_argument("--schedule", choices=("fused", "two_pass"), default="fused")
     ap.add_argument("--no-e2e", action="store_true")
@@ -443,6 +443,39 @@ class DSAIndexer(Workload):
                 tokens * self.H * (128 * 3 + 4), f"tokens 0..{tokens - 1} of the [{self.T},{self.H}] indexer input")
 
 
+class DSAIndexerNVFP4(DSAIndexer):
+    """The same indexer input, NVFP4 per rotated 128-vector (codes, E4M3 block
+    scales, per-vector decode scales transposed)."""
+    name = "dsa_indexer_nvfp4"
+
+    def alg_bytes(self):
+        # BF16 in (2) + codes (0.5) + block scales (1/16) per element + a float per vector
+        return self.elements() * 2 + self.elements() // 2 + self.elements() // 16 + self.T * self.H * 4
+
+    def config(self):
+        return {"workload": f"DSA indexer prep, FP4: cat q_pe|q_nope BF16 [{self.T},{self.H},64]x2 -> H128 -> NVFP4 "
+                            f"per 128-vector, vector scales [{self.H},{self.T}]",
+                "l2": "flushed before every step (256 MiB write)"}
+
+    def alloc_outputs(self, torch):
+        return {"codes": torch.empty((self.T, self.H * 64), dtype=torch.uint8, device="cuda"),
+                "block_sf": torch.empty((self.T, self.H * 8), dtype=torch.uint8, device="cuda"),
+                "sdec": torch.empty((self.H, self.T), dtype=torch.float32, device="cuda")}
+
+    def call(self, inputs, out):
+        self.hq.hq_cat_rotate_nvfp4(inputs["pe"], self.H * 64, 64, inputs["nope"], self.H * 64, 64, self.T, self.H,
+                                    128, out["codes"], out["block_sf"], out["sdec"], self.hq.HQ_SCALE_TRANSPOSED,
+                                    self.T)
+
+    def oracle_sample(self, host, tokens=256):
+        import oracle
+        pe, nope = host["pe"][:tokens], host["nope"][:tokens]
+        return (lambda: oracle.cat_rotate_nvfp4(pe, nope, tokens, self.H, 128, scale_layout=oracle.TRANSPOSED,
+                                                scale_ld=tokens),
+                tokens * self.H * 128 * 2 + tokens * self.H * (64 + 8 + 4),
+                f"tokens 0..{tokens - 1} of the [{self.T},{self.H}] indexer input")
+
+
 class FP8Single(DSAIndexer):
     name = "fp8_single"
 
@@ -525,6 +558,7 @@ def make_workload(name: str, rank: int, schedule: str = "fused") -> Workload:
             "grouped_moe_row_rht": lambda: GroupedRowRHT(rank, schedule=schedule),
             "dense_nvfp4": lambda: DenseNVFP4(rank, schedule=schedule),
             "dsa_indexer": lambda: DSAIndexer(rank),
+            "dsa_indexer_nvfp4": lambda: DSAIndexerNVFP4(rank),
             "fp8_single": lambda: FP8Single(rank),
             "qmoe_bf16": lambda: QMoE(rank, swiglu=False),
             "qmoe_swiglu": lambda: QMoE(rank, swiglu=True)}[name]()
@@ -708,8 +742,8 @@ def run_ours(args, ranks: Ranks) -> None:
         del main, host_main
         torch.cuda.empty_cache()
         extras = {}
-        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4", "dsa_indexer", "qmoe_bf16",
-                     "qmoe_swiglu", "fp8_single"):
+        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4", "dsa_indexer",
+                     "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"):
             if name == args.workload:
                 continue
             r = measure(torch, hq, name, args, ranks, flush)

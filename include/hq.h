@@ -231,6 +231,39 @@ hq_status hq_cat_rotate_fp8(const void *a, int64_t a_row_stride, int a_width,
 size_t hq_cat_rotate_fp8_workspace_size(void);
 
 /*
+ * The DSA indexer prep with an NVFP4 output (the FP4 path [DSA] names as
+ * lacking the rotation; the pages give no FP4 format, the reading is the
+ * two-level NVFP4 scheme of hq_group_rht_quant with the 128-vector in place
+ * of a section): concat and optional rotation exactly as hq_cat_rotate_fp8,
+ * then for each vector (t, g) with rotated values y:
+ *   A = max |y| over the vector, S_enc = 2688 / A (1 when A is 0 or the
+ *   quotient is not finite); per block of 16 consecutive values
+ *   sf = E4M3((a_b / 6) * S_enc), code_i = E2M1(y_i * S_enc / sf) (0 when
+ *   sf == 0); saturating round-to-nearest-even conversions.
+ *
+ *  a, b, a_width, b_width, strides, M, G, hadamard_n, scale_layout,
+ *  scale_ld   as hq_cat_rotate_fp8.
+ *  codes      uint8 [M, G*64]: vector (t, g) at (t * G + g) * 64, two E2M1
+ *             codes per byte, element 2k in the low nibble.  16-byte aligned.
+ *  block_sf   uint8 [M, G*8] E4M3 block scales.
+ *  sdec       float, per vector 1 / S_enc, in the FP8 scales' layouts
+ *             ([M, G] or [G, scale_ld]).  4-byte aligned.
+ *  amax_opt   float, NULL or A per vector, in the same layout.
+ *  ws, ws_bytes  unused: hq_cat_rotate_nvfp4_workspace_size() is 0.
+ * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
+ *         HQ_ERR_CUDA.  Inputs must be finite.
+ */
+hq_status hq_cat_rotate_nvfp4(const void *a, int64_t a_row_stride, int a_width,
+                              const void *b, int64_t b_row_stride, int b_width,
+                              int64_t M, int G, int hadamard_n,
+                              uint8_t *codes, uint8_t *block_sf, float *sdec,
+                              int scale_layout, int64_t scale_ld, float *amax_opt,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes hq_cat_rotate_nvfp4 needs: 0 (none). */
+size_t hq_cat_rotate_nvfp4_workspace_size(void);
+
+/*
  * QMoE dynamic FP8 activation quantizer [QMOE]: each row of K_out values is
  * split into consecutive groups of 128; each group gets the FP8 rule above.
  *  mode     HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32 or HQ_ACT_SWIGLU_F32 (the value

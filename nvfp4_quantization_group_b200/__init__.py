@@ -31,7 +31,8 @@ HQ_MAX_SECTIONS = 256
 EXPORTED = (
     "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
     "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8",
-    "hq_cat_rotate_fp8_workspace_size", "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
+    "hq_cat_rotate_fp8_workspace_size", "hq_cat_rotate_nvfp4", "hq_cat_rotate_nvfp4_workspace_size",
+    "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
 )
 
 
@@ -74,6 +75,11 @@ def lib() -> ctypes.CDLL:
                                         P, P, c_int, i64, P, P, sz, P]
         L.hq_cat_rotate_fp8_workspace_size.restype = sz
         L.hq_cat_rotate_fp8_workspace_size.argtypes = []
+        L.hq_cat_rotate_nvfp4.restype = c_int
+        L.hq_cat_rotate_nvfp4.argtypes = [P, i64, c_int, P, i64, c_int, i64, c_int, c_int,
+                                          P, P, P, c_int, i64, P, P, sz, P]
+        L.hq_cat_rotate_nvfp4_workspace_size.restype = sz
+        L.hq_cat_rotate_nvfp4_workspace_size.argtypes = []
         L.hq_swiglu_fp8_k128.restype = c_int
         L.hq_swiglu_fp8_k128.argtypes = [c_int, P, i64, i64, P, P, P, P, sz, P]
         L.hq_swiglu_fp8_k128_workspace_size.restype = sz
@@ -162,6 +168,18 @@ def hq_cat_rotate_fp8_workspace_size() -> int:
     return int(lib().hq_cat_rotate_fp8_workspace_size())
 
 
+def hq_cat_rotate_nvfp4(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, codes, block_sf, sdec,
+                        scale_layout, scale_ld, amax_opt=None, stream=None) -> None:
+    _check(lib().hq_cat_rotate_nvfp4(_p(a), int(a_row_stride), int(a_width), _p(b), int(b_row_stride),
+                                     int(b_width), int(M), int(G), int(hadamard_n), _p(codes), _p(block_sf), _p(sdec),
+                                     int(scale_layout), int(scale_ld), _p(amax_opt), None, 0, _stream(stream)),
+           "hq_cat_rotate_nvfp4")
+
+
+def hq_cat_rotate_nvfp4_workspace_size() -> int:
+    return int(lib().hq_cat_rotate_nvfp4_workspace_size())
+
+
 def hq_swiglu_fp8_k128(mode, inp, M, K_out, out_fp8, scales, amax_opt=None, stream=None) -> None:
     _check(lib().hq_swiglu_fp8_k128(int(mode), _p(inp), int(M), int(K_out), _p(out_fp8), _p(scales),
                                     _p(amax_opt), None, 0, _stream(stream)), "hq_swiglu_fp8_k128")
@@ -232,6 +250,29 @@ def cat_rotate_fp8(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 12
     hq_cat_rotate_fp8(a, a.stride(0), aw, b, 0 if b is None else b.stride(0), bw, M, G, hadamard_n, codes,
                       scales, scale_layout, ld, amax, stream)
     return (codes, scales, amax) if want_amax else (codes, scales)
+
+
+def cat_rotate_nvfp4(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 128,
+                     scale_layout: int = HQ_SCALE_ROWMAJOR, scale_ld: int | None = None, want_amax: bool = False,
+                     stream=None) -> dict:
+    """a: BF16 [M, G, a_width], b: BF16 [M, G, b_width] or None -> dict with codes [M, G*64],
+    block_sf [M, G*8], sdec (per vector, the scales' layout) and, with want_amax, amax."""
+    M, G, aw = a.shape
+    bw = 0 if b is None else b.shape[-1]
+    dev = a.device
+    out = {"codes": torch.empty((M, G * 64), dtype=torch.uint8, device=dev),
+           "block_sf": torch.empty((M, G * 8), dtype=torch.uint8, device=dev)}
+    if scale_layout == HQ_SCALE_ROWMAJOR:
+        out["sdec"] = torch.empty((M, G), dtype=torch.float32, device=dev)
+        ld = G
+    else:
+        ld = M if scale_ld is None else scale_ld
+        out["sdec"] = torch.empty((G, ld), dtype=torch.float32, device=dev)
+    if want_amax:
+        out["amax"] = torch.empty_like(out["sdec"])
+    hq_cat_rotate_nvfp4(a, a.stride(0), aw, b, 0 if b is None else b.stride(0), bw, M, G, hadamard_n, out["codes"],
+                        out["block_sf"], out["sdec"], scale_layout, ld, out.get("amax"), stream)
+    return out
 
 
 def swiglu_fp8_k128(mode: int, inp: torch.Tensor, K_out: int, want_amax: bool = False, stream=None):

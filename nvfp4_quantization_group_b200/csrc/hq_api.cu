@@ -262,22 +262,22 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
 size_t hq_cat_rotate_fp8_workspace_size(void) { return 0; }
 size_t hq_swiglu_fp8_k128_workspace_size(void) { return 0; }
 
-hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, const void* b,
-                            int64_t b_row_stride, int b_width, int64_t M, int G, int hadamard_n,
-                            uint8_t* out_fp8, float* scales, int scale_layout, int64_t scale_ld, float* amax_opt,
-                            void* ws, size_t ws_bytes, void* stream) {
-    (void)ws;
-    (void)ws_bytes;
+// Both DSA entry points: argument checks, tiling, launch.  fp4: NVFP4 codes
+// [M, G*64] in `out`, block scales [M, G*8] in `sf`, per-vector decode
+// scales in `scales`; else FP8 codes [M, G*128] and group scales.
+static hq_status cat_rotate(const void* a, int64_t a_row_stride, int a_width, const void* b, int64_t b_row_stride,
+                            int b_width, int64_t M, int G, int hadamard_n, uint8_t* out, uint8_t* sf, float* scales,
+                            int scale_layout, int64_t scale_ld, float* amax_opt, void* stream, bool fp4) {
     if (hadamard_n != 0 && hadamard_n != 128) return HQ_ERR_UNSUPPORTED;
     if (scale_layout != HQ_SCALE_ROWMAJOR && scale_layout != HQ_SCALE_TRANSPOSED) return HQ_ERR_UNSUPPORTED;
     if (M < 0 || G <= 0 || a_width < 0 || b_width < 0 || a_width + b_width != 128) return HQ_ERR_SHAPE;
     if (M == 0) return HQ_OK;
-    if (!a || !out_fp8 || !scales || (b_width > 0 && !b)) return HQ_ERR_NULL;
+    if (!a || !out || !scales || (b_width > 0 && !b) || (fp4 && !sf)) return HQ_ERR_NULL;
     if (a_width % 8 || b_width % 8 || a_row_stride % 8 || b_row_stride % 8) return HQ_ERR_ALIGN;
     if (a_row_stride < (int64_t)G * a_width || (b_width > 0 && b_row_stride < (int64_t)G * b_width))
         return HQ_ERR_SHAPE;
     if (scale_layout == HQ_SCALE_TRANSPOSED && scale_ld < M) return HQ_ERR_SHAPE;
-    if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out_fp8) || !aligned4(scales) ||
+    if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out) || !aligned4(scales) ||
         !aligned4(amax_opt))
         return HQ_ERR_ALIGN;
     const DeviceInfo* dev = device_info();
@@ -294,7 +294,8 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     p.M = M;
     p.G = G;
     p.rotate = hadamard_n == 128;
-    p.out = out_fp8;
+    p.out = out;
+    p.sf = sf;
     p.scales = scales;
     p.amax = amax_opt;
     p.scale_layout = scale_layout;
@@ -308,8 +309,30 @@ hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, co
     const int64_t tiles = p.ntiles;
     const int64_t cap = (int64_t)dev->sms * (dev->cat_blocks_per_sm > 0 ? dev->cat_blocks_per_sm : 1);
     const int grid = (int)(tiles < cap ? tiles : cap);
-    launch_cat_rotate(p, grid, (cudaStream_t)stream);
+    launch_cat_rotate(p, grid, (cudaStream_t)stream, fp4);
     return launch_status();
+}
+
+hq_status hq_cat_rotate_fp8(const void* a, int64_t a_row_stride, int a_width, const void* b,
+                            int64_t b_row_stride, int b_width, int64_t M, int G, int hadamard_n,
+                            uint8_t* out_fp8, float* scales, int scale_layout, int64_t scale_ld, float* amax_opt,
+                            void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    return cat_rotate(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, out_fp8, nullptr,
+                      scales, scale_layout, scale_ld, amax_opt, stream, false);
+}
+
+size_t hq_cat_rotate_nvfp4_workspace_size(void) { return 0; }
+
+hq_status hq_cat_rotate_nvfp4(const void* a, int64_t a_row_stride, int a_width, const void* b,
+                              int64_t b_row_stride, int b_width, int64_t M, int G, int hadamard_n,
+                              uint8_t* codes, uint8_t* block_sf, float* sdec, int scale_layout, int64_t scale_ld,
+                              float* amax_opt, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    return cat_rotate(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, codes, block_sf, sdec,
+                      scale_layout, scale_ld, amax_opt, stream, true);
 }
 
 hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out, uint8_t* out_fp8,

@@ -166,6 +166,45 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
+
+// ------------------------------------------------------- NVFP4 block math
+// Global encode scale of a section (or vector): 2688 / A (6 * 448); 1 when A
+// is not positive (a computed amax is 0 at worst; a given one may be
+// negative or NaN) or the quotient is not finite.
+__device__ __forceinline__ float global_encode(float A) {
+    float S = __fdiv_rn(2688.0f, A);
+    if (!(A > 0.0f) || !isfinite(S)) S = 1.0f;
+    return S;
+}
+
+// E4M3 block scale of a 16-block: E4M3((a_b / 6) * S_enc); a_b >= 0.
+__device__ __forceinline__ uint32_t block_sf(float ab, float senc) {
+    return e4m3x2(__fmul_rn(div6_rn(ab), senc), 0.0f) & 0xFFu;
+}
+
+// Per-block encode factor S / value(sf), correctly rounded (0 for codes 0
+// and 127), from a table vr[code] = {value, -RN(1 / value)}; `slow` when S
+// is outside [2^-100, 2^100] (the remainders could leave the normal range).
+__device__ __forceinline__ float block_enc(const float2* vr, uint32_t sf, float S, bool slow) {
+    const float2 e = vr[sf];
+    if (slow) return e.x == 0.0f ? 0.0f : __fdiv_rn(S, e.x);
+    return div_rn_neg(-S, Recip{e.x, e.y});
+}
+__device__ __forceinline__ bool slow_scale(float S) { return !(S >= 7.8886091e-31f && S <= 1.2676506e30f); }
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// max |x| over 16 values, as a tree of depth 3 (max is exact: any order gives
+// the same value; a NaN is skipped)
+__device__ __forceinline__ float absmax16(const float (&x)[16]) {
+    const float a = max3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2])), b = max3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+    const float c = max3(fabsf(x[6]), fabsf(x[7]), fabsf(x[8])), d = max3(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
+    const float e = max3(fabsf(x[12]), fabsf(x[13]), fabsf(x[14]));
+    return max3(max3(a, b, c), max3(d, e, fabsf(x[15])), 0.0f);
+}
 }  // namespace hq
 
 namespace hq {

@@ -1,10 +1,15 @@
-// hq_fp8.cu -- FP8 E4M3 group quantizers for sm_100a.
+// hq_fp8.cu -- FP8 E4M3 group quantizers for sm_100a, and the FP4 variant
+// of the DSA indexer prep.
 //
-//  * cat_rotate_fp8_kernel: DSA indexer prep (TensorRT-LLM PR #15158, code
+//  * cat_rotate_kernel<false>: DSA indexer prep (TensorRT-LLM PR #15158, code
 //    flow "torch.cat -> rotate_activation -> fp8_quantize_1x128"): concat of
 //    the pe and nope parts of each (token, head) vector, 128-point Sylvester
 //    Hadamard rotation scaled by 1/sqrt(128), then one E4M3 group of 128
 //    with the scale rule of onnxruntime PR #33644.
+//  * cat_rotate_kernel<true>: the same concat and rotation, then NVFP4 per
+//    vector (the FP4 path the same PR names as lacking the rotation): the
+//    vector's amax gives its global encode scale, each 16-element block an
+//    E4M3 scale and E2M1 codes, as in the grouped NVFP4 cast.
 //  * k128_fp8_kernel: QMoE dynamic FP8 activations (onnxruntime PR #33644,
 //    Description): consecutive K128 groups of BF16/FP32 rows, or of the FP32
 //    SwiGLU product SiLU(gate) * up.
@@ -147,9 +152,19 @@ __device__ __forceinline__ void cat_load(const CatRotateParams& p, CatVec cv, in
     }
 }
 
-__global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_fp8_kernel(CatRotateParams p) {
+template <bool FP4>
+__global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(CatRotateParams p) {
     __shared__ CatShared sh;
+    __shared__ float2 vr[FP4 ? 128 : 1];  // FP4: per E4M3 code {value, -RN(1 / value)}
     const int tid = threadIdx.x, k = tid >> 3, j = tid & 7;
+    if constexpr (FP4) {
+        if (tid < 128) {
+            const bool z = tid == 0 || tid == 127;
+            const float v = z ? 0.0f : e4m3_value((uint32_t)tid);
+            vr[tid] = make_float2(v, z ? -0.0f : -__frcp_rn(v));
+        }
+        __syncthreads();
+    }
     const float neg_c128 = -__uint_as_float(0x3DB504F3u);  // -RN(1/sqrt(128)): negated numerators
     const bf16_t minus_one = (bf16_t)0xBF80u;
 
@@ -235,6 +250,47 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_fp8_kerne
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
+        if constexpr (FP4) {
+            // ---- NVFP4: back to one 16-element block per thread (pair j of
+            // segment s at position (j + s) & 7 of the segment: both sides
+            // free of bank conflicts), then block scale and codes
+            const float S = global_encode(amax);
+            __syncwarp();  // the first exchange is read
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                float a, b;
+                unpack2(z[s], a, b);
+                sh.t[k][8 * s + ((j + s) & 7)] = make_float2(-a, -b);  // y = -z exactly
+            }
+            __syncwarp();
+            float y[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float2 e = sh.t[k][8 * j + ((i + j) & 7)];
+                y[2 * i] = e.x;
+                y[2 * i + 1] = e.y;
+            }
+            const uint32_t sf = block_sf(absmax16(y), S);
+            const float enc = block_enc(vr, sf, S, slow_scale(S));
+            const f2 e2 = pack2(enc, enc);
+            float q[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) unpack2(mul2(pack2(y[2 * i], y[2 * i + 1]), e2), q[2 * i], q[2 * i + 1]);
+            if (cv.t >= 0) {
+                const int64_t v = (int64_t)cv.t * p.G + cv.g;
+                *reinterpret_cast<uint2*>(p.out + v * 64 + 8 * j) =
+                    make_uint2(e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]),
+                               e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]));
+                p.sf[v * 8 + j] = (uint8_t)sf;
+                if (j == 0) {
+                    const int64_t si = p.scale_layout == 0 ? v : (int64_t)cv.g * p.scale_ld + cv.t;
+                    p.scales[si] = __fdiv_rn(1.0f, S);
+                    if (p.amax) p.amax[si] = amax;
+                }
+            }
+            __syncwarp();  // the exchange buffer is reused by the next tile
+            continue;
+        }
         const float sc = fp8_group_scale(amax);
         // ---- codes of elements 16s + 2j, 16s + 2j + 1
         uint32_t q[8];
@@ -431,13 +487,19 @@ int64_t cat_rotate_tiles(const CatRotateParams& p) {
 }
 
 int cat_rotate_blocks_per_sm() {
-    int n = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, cat_rotate_fp8_kernel, CAT_THREADS, 0);
+    // both variants: the grid is sized for the one with fewer resident CTAs
+    int n0 = 0, n1 = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, cat_rotate_kernel<false>, CAT_THREADS, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, cat_rotate_kernel<true>, CAT_THREADS, 0);
+    const int n = n0 < n1 ? n0 : n1;
     return n > 0 ? n : 1;
 }
 
-void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st) {
-    cat_rotate_fp8_kernel<<<grid, CAT_THREADS, 0, st>>>(p);
+void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st, bool fp4) {
+    if (fp4)
+        cat_rotate_kernel<true><<<grid, CAT_THREADS, 0, st>>>(p);
+    else
+        cat_rotate_kernel<false><<<grid, CAT_THREADS, 0, st>>>(p);
 }
 
 template <bool AMAX>

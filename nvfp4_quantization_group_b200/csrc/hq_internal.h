@@ -25,8 +25,9 @@ struct CatRotateParams {
     int wide;              // 16-element segments never straddle a and b, 32-byte aligned: 32-byte loads
     int G;
     int rotate;    // 1: H128 / sqrt(128); 0: none
-    uint8_t* out;
-    float* scales;
+    uint8_t* out;     // FP8: codes [M, G*128]; FP4: E2M1 codes [M, G*64]
+    float* scales;    // FP8: group scales; FP4: per-vector decode scales (1 / S_enc)
+    uint8_t* sf;      // FP4: E4M3 block scales [M, G*8]
     float* amax;  // NULL or per-group amax, in the scales' layout
     int scale_layout;
     int64_t scale_ld;
@@ -48,7 +49,7 @@ constexpr int K128_UNROLL = 4;      // warp steps with loads in flight
 int cat_rotate_blocks_per_sm();
 int64_t cat_rotate_tiles(const CatRotateParams& p);
 int cat_rotate_group_tiles(int G);  // group tiles of the transposed-scale layout
-void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st);
+void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st, bool fp4);
 void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st);
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st);
 

@@ -99,20 +99,6 @@ struct NvShared {
 // swizzle pattern is defined on 1024-byte aligned addresses)
 constexpr int NV_DYN_SMEM = NST * TILE_BYTES + (int)sizeof(NvShared) + 1024;
 
-// Section encode scale: 2688 / A (6 * 448); 1 when A is not positive (a
-// computed amax is 0 at worst; a given one may be negative or NaN) or the
-// quotient is not finite.
-__device__ __forceinline__ float global_encode(float A) {
-    float S = __fdiv_rn(2688.0f, A);
-    if (!(A > 0.0f) || !isfinite(S)) S = 1.0f;
-    return S;
-}
-
-// E4M3 block scale of a 16-block: E4M3((a_b / 6) * S_enc); t >= 0.
-__device__ __forceinline__ uint32_t block_sf(float ab, float senc) {
-    return e4m3x2(__fmul_rn(div6_rn(ab), senc), 0.0f) & 0xFFu;
-}
-
 __device__ __forceinline__ uint32_t hmax_abs(uint32_t a, uint32_t b) {
     uint32_t m;
     asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
@@ -181,20 +167,6 @@ __device__ __forceinline__ void row_rht(const uint32_t (&wa)[8], const uint32_t 
         v[2 * c + 1] = pack2(fma_bf16(a0, sg[2 * c], -pa), fma_bf16(b0, sg[2 * c], -pb));
     }
     rht_stages(v);
-}
-
-__device__ __forceinline__ float max3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-// max |x| over 16 values, as a tree of depth 3 (max is exact: any order gives
-// the same value)
-__device__ __forceinline__ float absmax16(const float (&x)[16]) {
-    const float a = max3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2])), b = max3(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
-    const float c = max3(fabsf(x[6]), fabsf(x[7]), fabsf(x[8])), d = max3(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
-    const float e = max3(fabsf(x[12]), fabsf(x[13]), fabsf(x[14]));
-    return max3(max3(a, b, c), max3(d, e, fabsf(x[15])), 0.0f);
 }
 
 // Shared byte offset of 16-byte chunk q (0..7) of column half h of tile row
@@ -292,14 +264,6 @@ __device__ __forceinline__ void red_max_u32(uint32_t* q, uint32_t v) {
 __device__ __forceinline__ void red_release_add_u32(uint32_t* q, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" :: "l"(q), "r"(v) : "memory");
 }
-// Per-block encode factor S / value(sf), correctly rounded (0 for codes 0
-// and 127); `slow` when S is outside [2^-100, 2^100].
-__device__ __forceinline__ float block_enc(const NvShared& sh, uint32_t sf, float S, bool slow) {
-    const float2 vr = sh.vr[sf];
-    if (slow) return vr.x == 0.0f ? 0.0f : __fdiv_rn(S, vr.x);
-    return div_rn_neg(-S, Recip{vr.x, vr.y});
-}
-__device__ __forceinline__ bool slow_scale(float S) { return !(S >= 7.8886091e-31f && S <= 1.2676506e30f); }
 
 // ---------------------------------------------------------------- producer
 // Producer state that persists across buffer fills.
@@ -486,8 +450,8 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const uint32_t code = (uint32_t)lane + 32u * m;
-                sh.enc[ps.tab][0][code] = block_enc(sh, code, ps.r_srq, fl & H_SLOW_R);
-                sh.enc[ps.tab][1][code] = block_enc(sh, code, ps.r_scq, fl & H_SLOW_C);
+                sh.enc[ps.tab][0][code] = block_enc(sh.vr, code, ps.r_srq, fl & H_SLOW_R);
+                sh.enc[ps.tab][1][code] = block_enc(sh.vr, code, ps.r_scq, fl & H_SLOW_C);
             }
             sh.tab_section[ps.tab] = t.s;  // (each lane reads back only its own write)
         }

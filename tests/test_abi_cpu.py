@@ -104,6 +104,24 @@ def test_cat_rotate_fp8_argument_errors(L):
     assert L.hq_cat_rotate_fp8_workspace_size() == 0
 
 
+def test_cat_rotate_nvfp4_argument_errors(L):
+    def call(a=FAKE, a_rs=64 * 64, aw=64, b=FAKE, b_rs=64 * 64, bw=64, M=16, G=64, hn=128, codes=FAKE, sf=FAKE,
+             sc=FAKE, layout=0, ld=16, amax=None):
+        return L.hq_cat_rotate_nvfp4(P(a), a_rs, aw, P(b), b_rs, bw, M, G, hn, P(codes), P(sf), P(sc), layout, ld,
+                                     P(amax), None, 0, None)
+    assert call(hn=16) == hq.HQ_ERR_UNSUPPORTED
+    assert call(layout=3) == hq.HQ_ERR_UNSUPPORTED
+    assert call(aw=64, bw=16) == hq.HQ_ERR_SHAPE
+    assert call(M=0) == hq.HQ_OK
+    assert call(sf=0) == hq.HQ_ERR_NULL
+    assert call(codes=0) == hq.HQ_ERR_NULL
+    assert call(sc=0) == hq.HQ_ERR_NULL
+    assert call(codes=FAKE + 8) == hq.HQ_ERR_ALIGN
+    assert call(amax=FAKE + 2) == hq.HQ_ERR_ALIGN
+    assert call(layout=1, ld=8) == hq.HQ_ERR_SHAPE
+    assert L.hq_cat_rotate_nvfp4_workspace_size() == 0
+
+
 def test_swiglu_fp8_k128_argument_errors(L):
     def call(mode=0, inp=FAKE, M=4, K=256, out=FAKE, sc=FAKE, amax=None):
         return L.hq_swiglu_fp8_k128(mode, P(inp), M, K, P(out), P(sc), P(amax), None, 0, None)

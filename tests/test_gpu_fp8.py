@@ -90,6 +90,66 @@ def test_dsa_indexer_full_4096x64(hq):
     _cat_case(hq, pe, nope, 4096, 64, 128, oracle.TRANSPOSED, ld=4096)
 
 
+# ------------------------------------------------------- cat -> H128 -> NVFP4
+from _compare import assert_fp4_codes  # noqa: E402
+
+
+def _cat4_case(hq, pe, nope, M, G, hadamard_n, layout, ld=None):
+    a = _dev(pe)
+    b = None if nope is None else _dev(nope)
+    got = hq.cat_rotate_nvfp4(a, b, hadamard_n, layout, ld, want_amax=True)
+    torch.cuda.synchronize()
+    got = {k: v.cpu().numpy() for k, v in got.items()}
+    want = oracle.cat_rotate_nvfp4(pe, nope, M, G, hadamard_n, scale_layout=layout,
+                                   scale_ld=ld if layout else None, want_amax=True)
+    for k in ("sdec", "amax"):
+        g, w = got[k], want[k]
+        if layout == oracle.TRANSPOSED:
+            g, w = g[:, :M], w[:, :M]
+        assert_bits_equal(g, w, k)
+    assert_bits_equal(got["block_sf"], want["block_sf"], "block_sf")
+    assert_fp4_codes(got["codes"], want["codes"],
+                     lambda: oracle.cat_rotate_nvfp4(pe, nope, M, G, hadamard_n, want_pre=True)["pre"], "fp4 codes")
+
+
+@pytest.mark.parametrize("hadamard_n", [0, 128])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_cat_nvfp4_ragged_tokens_and_heads(hq, hadamard_n, layout):
+    M, G = 37, 5
+    pe = S.normal_bf16(241, (M, G, 64))
+    nope = S.with_outliers_bf16(S.normal_bf16(242, (M, G, 64)), 243, p=0.01)
+    _cat4_case(hq, pe, nope, M, G, hadamard_n, layout, ld=40 if layout else None)
+
+
+def test_cat_nvfp4_zero_constant_and_single_tensor(hq):
+    M, G = 3, 2
+    pe = np.zeros((M, G, 64), dtype=np.uint16)
+    nope = np.zeros((M, G, 64), dtype=np.uint16)
+    pe[1] = S.f32_to_bf16_bits(np.full((G, 64), 1.5, np.float32))
+    nope[2, 1, 7] = S.f32_to_bf16_bits(np.float32([-3.0]))[0]
+    _cat4_case(hq, pe, nope, M, G, 128, oracle.ROWMAJOR)
+    _cat4_case(hq, pe, nope, M, G, 0, oracle.ROWMAJOR)
+    x = S.normal_bf16(251, (512, 1, 128))
+    _cat4_case(hq, x, None, 512, 1, 128, oracle.ROWMAJOR)
+
+
+def test_cat_nvfp4_magnitudes(hq):
+    """Vectors from 1e-30 to 1e30 (the slow encode path near the ends)."""
+    M, G = 8, 4
+    xf = S.bf16_bits_to_f32(S.normal_bf16(261, (M, G, 128))).copy()
+    xf *= np.float32(10.0) ** np.arange(-30, 34, 8, dtype=np.float32)[:, None, None]
+    x = S.f32_to_bf16_bits(xf)
+    _cat4_case(hq, x[..., :64].copy(), x[..., 64:].copy(), M, G, 128, oracle.TRANSPOSED, ld=8)
+
+
+@pytest.mark.slow
+def test_dsa_indexer_nvfp4_full_4096x64(hq):
+    seed = S.SEEDS["dsa_indexer"]
+    pe = S.normal_bf16(seed, (4096, 64, 64))
+    nope = S.normal_bf16(seed + 100, (4096, 64, 64))
+    _cat4_case(hq, pe, nope, 4096, 64, 128, oracle.TRANSPOSED, ld=4096)
+
+
 # ------------------------------------------------------------------ K128
 def _k128_case(hq, mode, x, M, K_out):
     codes, scales, amax = hq.swiglu_fp8_k128(mode, _dev(x), K_out, want_amax=True)
