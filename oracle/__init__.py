@@ -70,6 +70,14 @@ def lib() -> ctypes.CDLL:
             L.hqo_group_rht_quant.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_uint16, ctypes.c_uint,
                                               P, P, P, P, P, P, P, P, P, P]
             L.hqo_group_rht_quant.restype = ctypes.c_int
+            u64 = ctypes.c_uint64
+            L.hqo_group_rht_quant_sr.argtypes = [P, i64, i64, P, ctypes.c_int, ctypes.c_uint16, ctypes.c_uint,
+                                                 u64, u64, P, P, P, P, P, P, P, P, P, P]
+            L.hqo_group_rht_quant_sr.restype = ctypes.c_int
+            L.hqo_philox4x32_10.argtypes = [P, P, P]
+            L.hqo_philox4x32_10.restype = None
+            L.hqo_e2m1_sr_array.argtypes = [P, P, P, i64]
+            L.hqo_e2m1_sr_array.restype = None
             _lib = L
     return _lib
 
@@ -213,15 +221,34 @@ def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False, want_amax=False):
     return (out, scales, pre, amax) if want_amax else (out, scales, pre)
 
 
-ROWWISE, COLWISE, ROW_RHT, AMAX_GIVEN = 1, 2, 4, 16
+ROWWISE, COLWISE, ROW_RHT, AMAX_GIVEN, ROW_SR, COL_SR = 1, 2, 4, 16, 32, 64
+
+
+def e2m1_sr(t, r):
+    """Stochastic E2M1 codes of FP32 values t with random bytes r."""
+    t = np.ascontiguousarray(t, dtype=np.float32)
+    r = np.ascontiguousarray(r, dtype=np.uint8)
+    out = np.empty(t.shape, dtype=np.uint8)
+    lib().hqo_e2m1_sr_array(_ptr(t), _ptr(r), _ptr(out), t.size)
+    return out
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of a 4-word counter and a 2-word key -> 4 uint32."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.empty(4, dtype=np.uint32)
+    lib().hqo_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
 
 
 def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=False, amax_row=None,
-                    amax_col=None):
+                    amax_col=None, seed=0, offset=0):
     """Grouped RHT16 + NVFP4 cast.  x: uint16 BF16 bits [M, K].
 
     ROW_RHT (with ROWWISE) rotates every 16-element row block along K before
-    the rowwise amax and cast.  AMAX_GIVEN takes the section amax values from
+    the rowwise amax and cast.  ROW_SR / COL_SR round that direction's codes
+    stochastically with the random streams of seed / seed + 1 from offset.  AMAX_GIVEN takes the section amax values from
     amax_row / amax_col (float [S]) instead of computing them.
 
     Returns a dict with row_codes [M, K/2], row_sf [M, K/16], col_codes
@@ -254,7 +281,7 @@ def group_rht_quant(x, split_rows, sign_mask, flags=ROWWISE | COLWISE, want_pre=
         if flags & COLWISE:
             r["amax_col"][:] = np.asarray(amax_col, dtype=np.float32)
     g = r.get
-    rc = lib().hqo_group_rht_quant(_ptr(x), M, K, _ptr(splits), S, sign_mask, flags,
+    rc = lib().hqo_group_rht_quant_sr(_ptr(x), M, K, _ptr(splits), S, sign_mask, flags, seed, offset,
                                    _ptr(g("row_codes")), _ptr(g("row_sf")), _ptr(g("col_codes")),
                                    _ptr(g("col_sf")), _ptr(g("amax_row")), _ptr(g("amax_col")),
                                    _ptr(g("sdec_row")), _ptr(g("sdec_col")), _ptr(g("row_pre")),

@@ -387,10 +387,84 @@ static float global_encode_scale(float A)
     return S;
 }
 
+/* ------------------------------------------------ stochastic rounding */
+/*
+ * Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw,
+ * "Parallel random numbers: as easy as 1, 2, 3", SC 2011): ten rounds of
+ * the 4x32 Philox bijection on the counter, the key bumped by the Weyl
+ * increments before every round but the first.  A round maps
+ * (c0, c1, c2, c3) to (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1,
+ * lo(M0 c0)) with the paper's multipliers M0, M1.
+ */
+void hqo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;  /* multipliers */
+    const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;  /* Weyl increments of the key */
+    uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t p0 = (uint64_t)M0 * c[0], p1 = (uint64_t)M1 * c[2];
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c[1] ^ k0, n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c[3] ^ k1, n3 = (uint32_t)p0;
+        c[0] = n0;
+        c[1] = n1;
+        c[2] = n2;
+        c[3] = n3;
+    }
+    for (int i = 0; i < 4; ++i)
+        out[i] = c[i];
+}
+
+/* Byte `pos` of the random byte stream of `seed`: the little-endian bytes of
+ * the 32-bit words w_i = word (i mod 4) of Philox4x32-10(counter = i / 4 as
+ * a 64-bit number in the two low words, key = seed's two halves). */
+static uint8_t sr_byte(uint64_t seed, uint64_t pos)
+{
+    const uint64_t blk = pos / 16;
+    const uint32_t ctr[4] = {(uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    hqo_philox4x32_10(ctr, key, out);
+    return (uint8_t)(out[(pos % 16) / 4] >> (8 * (pos % 4)));
+}
+
+/* E2M1 code of t by stochastic rounding with the random byte r: |t| rounds up
+ * to the next E2M1 value iff r < floor(256 * f), f the fraction of |t| above
+ * the value below it in units of the grid step there (0.5 below 2, 1 below
+ * 4, 2 below 6); |t| >= 6 (and NaN) saturate to 6; the sign is kept, zero
+ * included (reading: the pages name stochastic rounding but give no rule). */
+static uint8_t e2m1_sr(float t, uint8_t r)
+{
+    const uint8_t sign = signbit(t) ? 8 : 0;
+    const float a = fabsf(t);
+    if (!(a < 6.0f))
+        return sign | 7;
+    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    const float q = a / step;      /* exact: a power-of-two step */
+    const float n = floorf(q);
+    const float f = q - n;         /* exact */
+    const unsigned F = (unsigned)(f * 256.0f);   /* floor: f * 256 < 256 */
+    const unsigned kk = (unsigned)n + (r < F ? 1u : 0u);
+    return sign | (uint8_t)(step == 0.5f ? kk : (step == 1.0f ? kk + 2u : kk + 4u));
+}
+
+/* e2m1_sr over arrays (for the pins). */
+void hqo_e2m1_sr_array(const float *t, const uint8_t *r, uint8_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e2m1_sr(t[i], r[i]);
+}
+
 /* Quantize one block of 16 values; codes packed two per byte, element 2k in
  * the low nibble and 2k+1 in the high nibble (reading: the pages are silent
- * on the packing). */
-static void nvfp4_block(const float *v, float S_enc, uint8_t *codes8, uint8_t *sf_out, float *pre)
+ * on the packing).  rnd, when given, holds the 16 random bytes of stochastic
+ * rounding; else round to nearest even. */
+static void nvfp4_block_r(const float *v, float S_enc, uint8_t *codes8, uint8_t *sf_out, float *pre,
+                          const uint8_t *rnd)
 {
     float ab = 0.0f;
     for (int i = 0; i < 16; ++i)
@@ -404,9 +478,16 @@ static void nvfp4_block(const float *v, float S_enc, uint8_t *codes8, uint8_t *s
             pre[2 * k] = t0;
             pre[2 * k + 1] = t1;
         }
-        codes8[k] = (uint8_t)((hqo_e2m1_encode(t0) & 0xF) | ((hqo_e2m1_encode(t1) & 0xF) << 4));
+        const uint8_t q0 = rnd ? e2m1_sr(t0, rnd[2 * k]) : (uint8_t)(hqo_e2m1_encode(t0) & 0xF);
+        const uint8_t q1 = rnd ? e2m1_sr(t1, rnd[2 * k + 1]) : (uint8_t)(hqo_e2m1_encode(t1) & 0xF);
+        codes8[k] = (uint8_t)(q0 | (q1 << 4));
     }
     *sf_out = sf;
+}
+
+static void nvfp4_block(const float *v, float S_enc, uint8_t *codes8, uint8_t *sf_out, float *pre)
+{
+    nvfp4_block_r(v, S_enc, codes8, sf_out, pre, 0);
 }
 
 /* The 16-point random Hadamard transform of [GRP]/[FUS]: v = 0.25 * H16 *
@@ -444,15 +525,24 @@ static void rht16(const float *x, uint16_t sign_mask, float *v)
  *   from the given A, and sdec_*[s] = 1/S_enc(A) for every section, empty
  *   ones included.  The pages do not describe this mode: it is the one-pass
  *   cast that a known amax allows, checked here by its definition.
+ * flags bit 5 / bit 6 (stochastic rounding, rowwise / columnwise; P2
+ *   discusses the Philox generator and deterministic offsets of TE's
+ *   stochastic rounding for this cast but gives no rule): the E2M1 codes of
+ *   that direction round stochastically (e2m1_sr) with random byte
+ *   offset + e of the stream of seed (rowwise) or seed + 1 (columnwise), e
+ *   the element's index in its output (r*K + c rowwise; the index inside
+ *   col_codes' element order columnwise).  Block scales stay nearest-even.
  * row_pre / col_pre, when given, receive the value rounded to E2M1 per
  * element, in the output's layout.
  */
-int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
-                        const int64_t *split_rows, int S, uint16_t sign_mask, unsigned flags,
-                        uint8_t *row_codes, uint8_t *row_sf, uint8_t *col_codes, uint8_t *col_sf,
-                        float *amax_row, float *amax_col, float *sdec_row, float *sdec_col,
-                        float *row_pre, float *col_pre)
+int hqo_group_rht_quant_sr(const uint16_t *x, int64_t M, int64_t K,
+                           const int64_t *split_rows, int S, uint16_t sign_mask, unsigned flags,
+                           uint64_t seed, uint64_t offset,
+                           uint8_t *row_codes, uint8_t *row_sf, uint8_t *col_codes, uint8_t *col_sf,
+                           float *amax_row, float *amax_col, float *sdec_row, float *sdec_col,
+                           float *row_pre, float *col_pre)
 {
+    uint8_t rnd[16];
     if (K % 128 != 0 || S < 0)
         return -1;
     int64_t total = 0;
@@ -494,9 +584,12 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                         blk[i] = bf16_value(x[r * K + kb * 16 + i]);
                     if (rotate)
                         rht16(blk, sign_mask, v);
-                    nvfp4_block(rotate ? v : blk, S_enc, row_codes + r * (K / 2) + kb * 8,
-                                row_sf + r * (K / 16) + kb,
-                                row_pre ? row_pre + r * K + kb * 16 : 0);
+                    if (flags & 32)  /* element r*K + c of the rowwise output: stream of seed */
+                        for (int i = 0; i < 16; ++i)
+                            rnd[i] = sr_byte(seed, offset + (uint64_t)(r * K + kb * 16 + i));
+                    nvfp4_block_r(rotate ? v : blk, S_enc, row_codes + r * (K / 2) + kb * 8,
+                                  row_sf + r * (K / 16) + kb,
+                                  row_pre ? row_pre + r * K + kb * 16 : 0, (flags & 32) ? rnd : 0);
                 }
         }
         if (flags & 2) {
@@ -523,8 +616,11 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
                     for (int i = 0; i < 16; ++i)
                         blk[i] = bf16_value(x[(r0 + mb * 16 + i) * K + c]);
                     rht16(blk, sign_mask, v);
-                    nvfp4_block(v, S_enc, cc + c * (Ms / 2) + mb * 8, cs + c * (Ms / 16) + mb,
-                                col_pre ? col_pre + K * r0 + c * Ms + mb * 16 : 0);
+                    if (flags & 64)  /* element of col_codes: stream of seed + 1 */
+                        for (int i = 0; i < 16; ++i)
+                            rnd[i] = sr_byte(seed + 1, offset + (uint64_t)(K * r0 + c * Ms + mb * 16 + i));
+                    nvfp4_block_r(v, S_enc, cc + c * (Ms / 2) + mb * 8, cs + c * (Ms / 16) + mb,
+                                  col_pre ? col_pre + K * r0 + c * Ms + mb * 16 : 0, (flags & 64) ? rnd : 0);
                 }
         }
         if (Ms == 0 && !given) {
@@ -534,6 +630,17 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
         r0 += Ms;
     }
     return 0;
+}
+
+/* hqo_group_rht_quant_sr with seed and offset 0. */
+int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
+                        const int64_t *split_rows, int S, uint16_t sign_mask, unsigned flags,
+                        uint8_t *row_codes, uint8_t *row_sf, uint8_t *col_codes, uint8_t *col_sf,
+                        float *amax_row, float *amax_col, float *sdec_row, float *sdec_col,
+                        float *row_pre, float *col_pre)
+{
+    return hqo_group_rht_quant_sr(x, M, K, split_rows, S, sign_mask, flags, 0, 0, row_codes, row_sf, col_codes,
+                                  col_sf, amax_row, amax_col, sdec_row, sdec_col, row_pre, col_pre);
 }
 
 /* ------------------------------------------------------------ FP4 DSA */

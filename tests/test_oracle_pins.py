@@ -658,6 +658,93 @@ def test_fp4_dsa_rotation_and_layouts():
     np.testing.assert_array_equal(rt["codes"], r["codes"])
 
 
+# ------------------------------------------------ stochastic rounding
+def _curand_words(seed, offset, n):
+    """cuRAND's host-side Philox4x32-10 generator (a library routine on the
+    CPU): n uint32 outputs of `seed` from output number `offset`."""
+    import ctypes
+    path = "/usr/local/cuda/lib64/libcurand.so"
+    if not os.path.exists(path):
+        pytest.skip("libcurand not present")
+    L = ctypes.CDLL(path)
+    L.curandSetPseudoRandomGeneratorSeed.argtypes = [ctypes.c_void_p, ctypes.c_ulonglong]
+    L.curandSetGeneratorOffset.argtypes = [ctypes.c_void_p, ctypes.c_ulonglong]
+    L.curandGenerate.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t]
+    g = ctypes.c_void_p()
+    assert L.curandCreateGeneratorHost(ctypes.byref(g), 161) == 0       # CURAND_RNG_PSEUDO_PHILOX4_32_10
+    assert L.curandSetPseudoRandomGeneratorSeed(g, seed) == 0
+    assert L.curandSetGeneratorOffset(g, offset) == 0
+    out = np.zeros(n, dtype=np.uint32)
+    assert L.curandGenerate(g, out.ctypes.data, n) == 0
+    L.curandDestroyGenerator(g)
+    return out
+
+
+@pytest.mark.parametrize("seed", [0, 1, 0x0123456789ABCDEF, 2**64 - 1])
+def test_philox_matches_curand_host_generator(seed):
+    """The oracle's Philox4x32-10 against cuRAND's host generator (a library
+    routine on the CPU).  Its output block i is Philox with counter
+    (i >> 16, 0, i & 0xFFFF, 0) and key = the seed's halves (observed layout
+    of its default ordering), which exercises counter words 0 and 2 and the
+    key; words 1 and 3 enter only through the same XORs as the key."""
+    for i in (0, 1, 65535, 65536, 65536 * 7 + 123, (1 << 47) + 5):
+        w = _curand_words(seed, 4 * i, 4)
+        got = oracle.philox4x32_10([i >> 16 & 0xFFFFFFFF, 0, i & 0xFFFF, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        np.testing.assert_array_equal(got, w, err_msg=f"block {i}")
+
+
+def test_e2m1_stochastic_rounding_rule():
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float32)
+    rb = np.arange(256, dtype=np.uint8)
+    # on the grid: the nearest-even code for every random byte, signs kept
+    for sgn in (1, -1):
+        t = np.repeat(sgn * grid, 256)
+        want = np.repeat(oracle.encode_array(oracle.E2M1, sgn * grid), 256)
+        np.testing.assert_array_equal(oracle.e2m1_sr(t, np.tile(rb, 8)), want & 0xF)
+    # between grid values: probability of rounding up = floor(256 f) / 256 exactly
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        i = int(rng.integers(0, 7))
+        lo, hi = float(grid[i]), float(grid[i + 1])
+        t = np.float32(lo + (hi - lo) * rng.random())
+        if t == lo or t >= 6:
+            continue
+        f = (Fraction(float(t)) - Fraction(lo)) / (Fraction(hi) - Fraction(lo))
+        F = int(f * 256)                                            # floor
+        codes = oracle.e2m1_sr(np.full(256, t), rb)
+        up = codes == oracle.e2m1_sr(np.array([hi], np.float32), np.zeros(1, np.uint8))[0]
+        assert int(up.sum()) == F and np.all(up == (rb < F))
+        assert oracle.e2m1_sr(np.array([-t]), np.array([0], np.uint8))[0] & 8        # sign kept
+    # beyond 6 (and at it): saturate
+    np.testing.assert_array_equal(oracle.e2m1_sr(np.array([6, 7, 1e30, -8], np.float32), np.zeros(4, np.uint8)),
+                                  np.array([7, 7, 7, 15], np.uint8))
+
+
+def test_stochastic_rounding_streams_of_the_grouped_cast():
+    """ROW_SR / COL_SR: each code is e2m1_sr of its pre-rounding value with
+    byte offset + e of the Philox byte stream of seed (rowwise) or seed + 1
+    (columnwise; counter = byte / 16 in the two low words), e the element's
+    index in its output; block scales and amax as without stochastic
+    rounding."""
+    x = S.normal_bf16(331, (256, 128))
+    splits, mask, seed, offset = [128, 128], 0x3A5C, 0x00FF00FF12345678, 4096
+    flags = oracle.ROWWISE | oracle.COLWISE
+    rn = oracle.group_rht_quant(x, splits, mask, flags)
+    r = oracle.group_rht_quant(x, splits, mask, flags | oracle.ROW_SR | oracle.COL_SR, want_pre=True,
+                               seed=seed, offset=offset)
+    for k in ("row_sf", "col_sf", "amax_row", "amax_col", "sdec_row", "sdec_col"):
+        np.testing.assert_array_equal(r[k], rn[k], err_msg=k)
+    n = 256 * 128
+    for d, key, pre in ((0, "row_codes", r["row_pre"]), (1, "col_codes", r["col_pre"])):
+        k = seed + d
+        blocks = [oracle.philox4x32_10([b & 0xFFFFFFFF, b >> 32, 0, 0], [k & 0xFFFFFFFF, k >> 32])
+                  for b in range(offset // 16, (offset + n) // 16)]
+        rbytes = np.concatenate(blocks).view(np.uint8)                 # little-endian bytes, from byte `offset`
+        want = oracle.e2m1_sr(pre.reshape(-1), rbytes)
+        np.testing.assert_array_equal(_unpack(r[key]).reshape(-1), want, err_msg=key)
+    assert not np.array_equal(r["col_codes"], rn["col_codes"])
+
+
 def test_nvfp4_zero_section_and_tiny_values():
     x = np.zeros((256, 128), dtype=np.uint16)
     x[128:] = S.normal_bf16(97, (128, 128))
