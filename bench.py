@@ -54,7 +54,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="grouped_moe",
-                    choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4",
+                    choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr", "dense_nvfp4",
                              "dsa_indexer", "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
     ap.add_argument("--no-extras", action="store_true", help="time only the headline workload")
     ap.add_argument("--schedule", choices=("fused", "two_pass"), default="fused")
@@ -387,6 +387,32 @@ class GroupedRowRHT(GroupedNVFP4):
                 f"one {rows}-row section of the BF16 [{self.M},{self.K}] input, rows rotated too")
 
 
+class GroupedSR(GroupedNVFP4):
+    """The same workload with stochastic rounding of both directions' codes
+    (hq_group_rht_quant_sr, Philox4x32-10 random bytes)."""
+    name = "grouped_moe_sr"
+
+    def config(self):
+        c = super().config()
+        c["workload"] += ", stochastic rounding (rowwise and columnwise codes)"
+        return c
+
+    def call(self, inputs, out):
+        hq = self.hq
+        hq.hq_group_rht_quant_sr(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask,
+                                 hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_ROW_SR | hq.HQ_COL_SR, 1234, 0,
+                                 out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
+                                 out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
+
+    def oracle_sample(self, host, rows=512):
+        import oracle
+        x = host["x"][:rows]
+        flags = oracle.ROWWISE | oracle.COLWISE | oracle.ROW_SR | oracle.COL_SR
+        return (lambda: oracle.group_rht_quant(x, [rows], self.mask, flags, seed=1234, offset=0),
+                rows * self.K * 2 + 2 * (rows * self.K // 2 + rows * self.K // 16),
+                f"one {rows}-row section of the BF16 [{self.M},{self.K}] input, stochastic rounding")
+
+
 class DenseNVFP4(GroupedNVFP4):
     name = "dense_nvfp4"
 
@@ -556,6 +582,7 @@ def make_workload(name: str, rank: int, schedule: str = "fused") -> Workload:
     return {"grouped_moe": lambda: GroupedNVFP4(rank, schedule=schedule),
             "grouped_moe_amax_given": lambda: GroupedAmaxGiven(rank),
             "grouped_moe_row_rht": lambda: GroupedRowRHT(rank, schedule=schedule),
+            "grouped_moe_sr": lambda: GroupedSR(rank, schedule=schedule),
             "dense_nvfp4": lambda: DenseNVFP4(rank, schedule=schedule),
             "dsa_indexer": lambda: DSAIndexer(rank),
             "dsa_indexer_nvfp4": lambda: DSAIndexerNVFP4(rank),
@@ -742,7 +769,7 @@ def run_ours(args, ranks: Ranks) -> None:
         del main, host_main
         torch.cuda.empty_cache()
         extras = {}
-        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "dense_nvfp4", "dsa_indexer",
+        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr", "dense_nvfp4", "dsa_indexer",
                      "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"):
             if name == args.workload:
                 continue

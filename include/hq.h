@@ -58,6 +58,8 @@ typedef enum hq_status {
 #define HQ_COLWISE 2u      /* columnwise NVFP4 output (RHT16 along M, transposed) */
 #define HQ_ROW_RHT 4u      /* with HQ_ROWWISE: the rowwise output casts the RHT16
                               of each 16-column block along K instead of x */
+#define HQ_ROW_SR 32u      /* hq_group_rht_quant_sr: rowwise codes round stochastically */
+#define HQ_COL_SR 64u      /* hq_group_rht_quant_sr: columnwise codes round stochastically */
 #define HQ_AMAX_GIVEN 16u  /* amax_row / amax_col are inputs: the caller's section
                               amax values; one pass, no amax computation */
 #define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
@@ -169,6 +171,33 @@ hq_status hq_group_rht_quant(const void *x, int64_t M, int64_t K,
                              float *amax_row, float *amax_col,
                              float *sdec_row, float *sdec_col,
                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * hq_group_rht_quant with stochastic rounding of the E2M1 codes (the grouped
+ * pages' review discusses the Philox generator and deterministic offsets of
+ * stochastic rounding for this cast; it gives no rounding rule).  flags may
+ * add HQ_ROW_SR (with HQ_ROWWISE) and HQ_COL_SR (with HQ_COLWISE); block
+ * scales, amax and sdec are as without.  A code rounds |v| (v = value *
+ * encode factor, as for nearest-even) up to the next E2M1 value iff its
+ * random byte r < floor(256 f), f the fraction of |v| above the E2M1 value
+ * below it in grid steps (0.5 below 2, 1 below 4, 2 below 6); |v| >= 6
+ * saturates; the sign is kept.  r of output element e (its index in
+ * row_codes' [M, K] order, or in col_codes' element order) is byte
+ * offset + e of the stream of bytes B_i = byte (i % 4) of word (i / 4) % 4
+ * of Philox4x32-10(counter = {i / 16 low 32 bits, i / 16 high 32 bits, 0, 0},
+ * key = {k low, k high}), k = seed for rowwise codes and seed + 1 for
+ * columnwise codes, so results depend only on (seed, offset), not on the
+ * launch.  offset must be a multiple of 16 (HQ_ERR_ALIGN).  Other arguments,
+ * outputs and errors as hq_group_rht_quant (which rejects the SR flags).
+ */
+hq_status hq_group_rht_quant_sr(const void *x, int64_t M, int64_t K,
+                                const int64_t *split_rows, int S, uint16_t sign_mask,
+                                unsigned flags, uint64_t seed, uint64_t offset,
+                                uint8_t *row_codes, uint8_t *row_sf,
+                                uint8_t *col_codes, uint8_t *col_sf,
+                                float *amax_row, float *amax_col,
+                                float *sdec_row, float *sdec_col,
+                                void *ws, size_t ws_bytes, void *stream);
 
 /*
  * hq_group_rht_quant without a caller workspace, for callers that cannot

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libhq.so")
 
 HQ_OK, HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE, HQ_ERR_UNSUPPORTED, HQ_ERR_CUDA, \
     HQ_ERR_TIMEOUT = range(8)
-HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS, HQ_AMAX_GIVEN = 1, 2, 4, 8, 16
+HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS, HQ_AMAX_GIVEN, HQ_ROW_SR, HQ_COL_SR = 1, 2, 4, 8, 16, 32, 64
 HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
 HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
 HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1
@@ -30,7 +30,7 @@ HQ_MAX_SECTIONS = 256
 
 EXPORTED = (
     "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
-    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8",
+    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_sr", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8",
     "hq_cat_rotate_fp8_workspace_size", "hq_cat_rotate_nvfp4", "hq_cat_rotate_nvfp4_workspace_size",
     "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
 )
@@ -67,6 +67,9 @@ def lib() -> ctypes.CDLL:
         L.hq_group_rht_quant.restype = c_int
         L.hq_group_rht_quant.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
                                          P, P, P, P, P, P, P, P, P, sz, P]
+        L.hq_group_rht_quant_sr.restype = c_int
+        L.hq_group_rht_quant_sr.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u, ctypes.c_uint64,
+                                            ctypes.c_uint64, P, P, P, P, P, P, P, P, P, sz, P]
         L.hq_group_rht_quant_noalloc.restype = c_int
         L.hq_group_rht_quant_noalloc.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
                                                  P, P, P, P, P, P, P, P, P]
@@ -145,6 +148,17 @@ def hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, row_codes, row_
                                     _p(sdec_col), _p(ws), ws_bytes, _stream(stream)), "hq_group_rht_quant")
 
 
+def hq_group_rht_quant_sr(x, M, K, split_rows, S, sign_mask, flags, seed, offset, row_codes, row_sf, col_codes,
+                          col_sf, amax_row, amax_col, sdec_row, sdec_col, ws, stream=None) -> None:
+    splits = (ctypes.c_int64 * len(split_rows))(*[int(v) for v in split_rows])
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().hq_group_rht_quant_sr(_p(x), int(M), int(K), ctypes.cast(splits, ctypes.c_void_p), int(S),
+                                       int(sign_mask) & 0xFFFF, int(flags), int(seed) & (2**64 - 1),
+                                       int(offset) & (2**64 - 1), _p(row_codes), _p(row_sf), _p(col_codes),
+                                       _p(col_sf), _p(amax_row), _p(amax_col), _p(sdec_row), _p(sdec_col), _p(ws),
+                                       ws_bytes, _stream(stream)), "hq_group_rht_quant_sr")
+
+
 def hq_group_rht_quant_noalloc(x, M, K, split_rows, S, sign_mask, flags, row_codes, row_sf, col_codes, col_sf,
                                amax_row, amax_col, sdec_row, sdec_col, stream=None) -> None:
     """hq_group_rht_quant with the library's fixed scratch array instead of a
@@ -218,8 +232,10 @@ def group_outputs(M: int, K: int, S: int, flags: int = HQ_ROWWISE | HQ_COLWISE, 
 
 
 def group_rht_quant(x: torch.Tensor, split_rows, sign_mask: int, flags: int = HQ_ROWWISE | HQ_COLWISE,
-                    ws: torch.Tensor | None = None, out: dict | None = None, stream=None) -> dict:
-    """Grouped RHT16 + NVFP4 cast of a BF16 [M, K] CUDA tensor (see hq.h)."""
+                    ws: torch.Tensor | None = None, out: dict | None = None, stream=None, seed: int | None = None,
+                    offset: int = 0) -> dict:
+    """Grouped RHT16 + NVFP4 cast of a BF16 [M, K] CUDA tensor (see hq.h); with a seed, through
+    hq_group_rht_quant_sr (stochastic rounding for HQ_ROW_SR / HQ_COL_SR)."""
     M, K = x.shape
     S = len(split_rows)
     if ws is None:
@@ -227,8 +243,13 @@ def group_rht_quant(x: torch.Tensor, split_rows, sign_mask: int, flags: int = HQ
     if out is None:
         out = group_outputs(M, K, S, flags, x.device)
     g = out.get
-    hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, g("row_codes"), g("row_sf"), g("col_codes"),
-                       g("col_sf"), g("amax_row"), g("amax_col"), g("sdec_row"), g("sdec_col"), ws, stream)
+    if seed is not None:
+        hq_group_rht_quant_sr(x, M, K, split_rows, S, sign_mask, flags, seed, offset, g("row_codes"), g("row_sf"),
+                              g("col_codes"), g("col_sf"), g("amax_row"), g("amax_col"), g("sdec_row"),
+                              g("sdec_col"), ws, stream)
+    else:
+        hq_group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, g("row_codes"), g("row_sf"), g("col_codes"),
+                           g("col_sf"), g("amax_row"), g("amax_col"), g("sdec_row"), g("sdec_col"), ws, stream)
     return out
 
 

@@ -124,12 +124,17 @@ hq_status hq_get_error(void* ws, size_t ws_bytes, uint32_t* err_out, void* strea
     return HQ_OK;
 }
 
-hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
-                             uint16_t sign_mask, unsigned flags, uint8_t* row_codes, uint8_t* row_sf,
-                             uint8_t* col_codes, uint8_t* col_sf, float* amax_row, float* amax_col,
-                             float* sdec_row, float* sdec_col, void* ws, size_t ws_bytes, void* stream) {
+static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
+                                 uint16_t sign_mask, unsigned flags, uint64_t sr_seed, uint64_t sr_offset,
+                                 uint8_t* row_codes, uint8_t* row_sf, uint8_t* col_codes, uint8_t* col_sf,
+                                 float* amax_row, float* amax_col, float* sdec_row, float* sdec_col, void* ws,
+                                 size_t ws_bytes, void* stream) {
     // ---- argument checks (nothing is launched on failure)
-    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS)) return HQ_ERR_UNSUPPORTED;
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR))
+        return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_ROW_SR) && !(flags & HQ_ROWWISE)) return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_COL_SR) && !(flags & HQ_COLWISE)) return HQ_ERR_UNSUPPORTED;
+    if (sr_offset % 16 != 0) return HQ_ERR_ALIGN;  // a 16-element block takes one random block
     const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
     if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
     if ((flags & HQ_ROW_RHT) && !do_row) return HQ_ERR_UNSUPPORTED;
@@ -168,7 +173,9 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     p.ws = static_cast<uint32_t*>(ws);
     p.S = S;
     p.sign_mask = sign_mask;
-    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN);
+    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_ROW_SR | HQ_COL_SR);
+    p.sr_seed = sr_seed;
+    p.sr_offset = sr_offset;
     p.col_tiles = (int)(K / NV_TILE);
     int row0 = 0;
     int live[HQ_MAX_SECTIONS];
@@ -257,6 +264,24 @@ hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t*
     hq_status r = launch(pa, na);
     if (r != HQ_OK) return r;
     return launch(pc, nc);
+}
+
+hq_status hq_group_rht_quant(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
+                             uint16_t sign_mask, unsigned flags, uint8_t* row_codes, uint8_t* row_sf,
+                             uint8_t* col_codes, uint8_t* col_sf, float* amax_row, float* amax_col,
+                             float* sdec_row, float* sdec_col, void* ws, size_t ws_bytes, void* stream) {
+    if (flags & (HQ_ROW_SR | HQ_COL_SR)) return HQ_ERR_UNSUPPORTED;  // needs a seed: hq_group_rht_quant_sr
+    return group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, 0, 0, row_codes, row_sf, col_codes, col_sf,
+                           amax_row, amax_col, sdec_row, sdec_col, ws, ws_bytes, stream);
+}
+
+hq_status hq_group_rht_quant_sr(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
+                                uint16_t sign_mask, unsigned flags, uint64_t seed, uint64_t offset,
+                                uint8_t* row_codes, uint8_t* row_sf, uint8_t* col_codes, uint8_t* col_sf,
+                                float* amax_row, float* amax_col, float* sdec_row, float* sdec_col, void* ws,
+                                size_t ws_bytes, void* stream) {
+    return group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, seed, offset, row_codes, row_sf, col_codes,
+                           col_sf, amax_row, amax_col, sdec_row, sdec_col, ws, ws_bytes, stream);
 }
 
 size_t hq_cat_rotate_fp8_workspace_size(void) { return 0; }

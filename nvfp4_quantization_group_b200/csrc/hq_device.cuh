@@ -197,6 +197,60 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
+// ----------------------------------------------------- stochastic rounding
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC 2011): ten rounds of
+//   (c0, c1, c2, c3) -> (hi(B c2) ^ c1 ^ k0, lo(B c2), hi(A c0) ^ c3 ^ k1, lo(A c0)),
+// with the paper's multipliers A, B, the key advanced by its Weyl
+// increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+    constexpr uint32_t A = 0xD2511F53u, B = 0xCD9E8D57u, WA = 0x9E3779B9u, WB = 0xBB67AE85u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += WA;
+            k1 += WB;
+        }
+        const uint32_t ha = __umulhi(A, c.x), la = A * c.x;
+        const uint32_t hb = __umulhi(B, c.z), lb = B * c.z;
+        c = make_uint4(hb ^ c.y ^ k0, lb, ha ^ c.w ^ k1, la);
+    }
+    return c;
+}
+
+// The 16 random bytes (four words, byte i of the block in byte i % 4 of word
+// i / 4) of 16-byte block `blk` of the stream of `seed`.
+__device__ __forceinline__ uint4 sr_block(uint64_t seed, uint64_t blk) {
+    return philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+}
+
+// E2M1 code (4 bits) of t by stochastic rounding with random byte r: |t| goes
+// up to the next E2M1 value iff r < floor(256 f), f the fraction of |t|
+// above the value below, in grid steps (0.5 below 2, 1 below 4, 2 below 6);
+// |t| >= 6 and NaN saturate to 6; the sign is kept, zero included.  (A
+// branch-free version on the integer bits measured 8 % slower, one with
+// branches 27 % slower.)
+__device__ __forceinline__ uint32_t e2m1_sr(float t, uint32_t r) {
+    const uint32_t sign = (__float_as_uint(t) >> 28) & 8u;
+    const float a = fabsf(t);
+    if (!(a < 6.0f)) return sign | 7u;
+    const bool b2 = a < 2.0f, b4 = a < 4.0f;
+    const float q = __fmul_rn(a, b2 ? 2.0f : (b4 ? 1.0f : 0.5f));  // in grid steps: exact
+    const float n = floorf(q);
+    const uint32_t F = __float2uint_rz(__fmul_rn(__fsub_rn(q, n), 256.0f));  // floor(256 f), exact operands
+    return sign | ((uint32_t)n + (r < F ? 1u : 0u) + (b2 ? 0u : (b4 ? 2u : 4u)));
+}
+
+// Eight stochastic E2M1 codes packed like e2m1x8 (element k in nibble k),
+// with the random bytes of word pair (w0: elements 0..3, w1: 4..7).
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float* v, uint32_t w0, uint32_t w1) {
+    uint32_t r = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) r |= e2m1_sr(v[k], ((k < 4 ? w0 : w1) >> (8 * (k & 3))) & 0xFFu) << (4 * k);
+    return r;
+}
+
 // max |x| over 16 values, as a tree of depth 3 (max is exact: any order gives
 // the same value; a NaN is skipped)
 __device__ __forceinline__ float absmax16(const float (&x)[16]) {

@@ -152,6 +152,8 @@ struct NvParams {
     int S;
     uint32_t sign_mask;
     uint32_t flags;
+    uint64_t sr_seed;    // stochastic rounding: stream keys (rowwise seed, columnwise seed + 1)
+    uint64_t sr_offset;  //   and the byte the streams start at (a multiple of 16)
     int col_tiles;      // K / 128
     int nseg;           // schedule segments
     uint32_t total_items;

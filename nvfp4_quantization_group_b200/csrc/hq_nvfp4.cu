@@ -506,7 +506,9 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
 
 // ------------------------------------------------------------ compute warps
 // RowRht: the rowwise blocks are rotated along K before their amax and cast.
-template <bool RowRht>
+// SR: the codes of the directions HQ_ROW_SR / HQ_COL_SR select round
+// stochastically (one Philox block per 16-element block).
+template <bool RowRht, bool SR>
 __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, const uint8_t* tiles, int w,
                                             int lane) {
     uint32_t* const err = p.ws + 2;
@@ -515,6 +517,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
     uint32_t* const amax_col_ws = amax_row_ws + p.S;
     uint32_t* const done_ws = amax_col_ws + p.S;
     const bool do_row = p.flags & HQ_ROWWISE, do_col = p.flags & HQ_COLWISE;
+    const bool sr_row = SR && (p.flags & HQ_ROW_SR), sr_col = SR && (p.flags & HQ_COL_SR);
 
     const uint8_t* T_cur = tiles;  // the buffer being worked on
     bf16_t sg[16];  // sigma_i as BF16 +-1
@@ -677,12 +680,22 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 #pragma unroll
                 for (int i = 0; i < 16; ++i) unpack2(mul2(v[i], e2), q0[i], q1[i]);
                 // rows rr and rr + 4: codes in element order (no chunk swap)
-                *reinterpret_cast<uint2*>(rc_base + 8u * pt.rs_off0) =
-                    make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
-                               e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
-                *reinterpret_cast<uint2*>(rc_base + 8u * (pt.rs_off0 + 4u * K16)) =
-                    make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
-                               e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
+                uint2 ca, cbw;
+                if (sr_row) {
+                    // element index of the block's first element in row_codes' order
+                    const uint64_t e0 = (uint64_t)h.row0 * (uint64_t)p.K + (uint32_t)h.col0 + 16u * pt.rs_off0;
+                    const uint4 wa = sr_block(p.sr_seed, (p.sr_offset + e0) / 16u);
+                    const uint4 wb = sr_block(p.sr_seed, (p.sr_offset + e0 + 64u * K16) / 16u);
+                    ca = make_uint2(e2m1x8_sr(q0, wa.x, wa.y), e2m1x8_sr(q0 + 8, wa.z, wa.w));
+                    cbw = make_uint2(e2m1x8_sr(q1, wb.x, wb.y), e2m1x8_sr(q1 + 8, wb.z, wb.w));
+                } else {
+                    ca = make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
+                                    e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
+                    cbw = make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
+                                     e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
+                }
+                *reinterpret_cast<uint2*>(rc_base + 8u * pt.rs_off0) = ca;
+                *reinterpret_cast<uint2*>(rc_base + 8u * (pt.rs_off0 + 4u * K16)) = cbw;
                 rs_base[pt.rs_off0] = (uint8_t)sf0;
                 rs_base[pt.rs_off0 + 4u * K16] = (uint8_t)sf1;
             } else if (do_row) {
@@ -704,9 +717,18 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                         split_bf16x2(wd[c], xl, xh);
                         unpack2(mul2(pack2(add_bf16(xl, -0.0f), add_bf16(xh, -0.0f)), e2), q[2 * c], q[2 * c + 1]);
                     }
-                    const uint32_t c0 = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-                    const uint32_t c1 = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
                     const uint64_t rs_off = pt.rs_off0 + (kk ? 4u * K16 : 0u);
+                    uint32_t c0, c1;
+                    if (sr_row) {
+                        const uint64_t e0 = (uint64_t)h.row0 * (uint64_t)p.K + (uint32_t)h.col0 + 16u * rs_off;
+                        const uint4 w4 = sr_block(p.sr_seed, (p.sr_offset + e0) / 16u);
+                        // q[0..7] are elements 8..15 of the block on lanes that loaded the odd chunk first
+                        c0 = e2m1x8_sr(q, swap ? w4.z : w4.x, swap ? w4.w : w4.y);
+                        c1 = e2m1x8_sr(q + 8, swap ? w4.x : w4.z, swap ? w4.y : w4.w);
+                    } else {
+                        c0 = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+                        c1 = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+                    }
                     *reinterpret_cast<uint2*>(rc_base + 8u * rs_off) =
                         swap ? make_uint2(c1, c0) : make_uint2(c0, c1);
                     rs_base[rs_off] = (uint8_t)sf;
@@ -740,12 +762,22 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                                     ((uint32_t)h.row_in_sec0 / 2u + 8u * (uint32_t)rb);
                 uint8_t* const sb = p.col_sf + (uint64_t)h.r0s * K16 + c * ms16 +
                                     ((uint32_t)h.row_in_sec0 / 16u + (uint32_t)rb);
-                *reinterpret_cast<uint2*>(cb) =
-                    make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
-                               e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
-                *reinterpret_cast<uint2*>(cb + ms2) =
-                    make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
-                               e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
+                if (sr_col) {
+                    // element index in col_codes' order: twice the byte offset of cb
+                    const uint64_t e0 = 2u * (uint64_t)(cb - p.col_codes);
+                    const uint4 wa = sr_block(p.sr_seed + 1u, (p.sr_offset + e0) / 16u);
+                    const uint4 wb = sr_block(p.sr_seed + 1u, (p.sr_offset + e0 + 2u * ms2) / 16u);
+                    *reinterpret_cast<uint2*>(cb) = make_uint2(e2m1x8_sr(q0, wa.x, wa.y), e2m1x8_sr(q0 + 8, wa.z, wa.w));
+                    *reinterpret_cast<uint2*>(cb + ms2) =
+                        make_uint2(e2m1x8_sr(q1, wb.x, wb.y), e2m1x8_sr(q1 + 8, wb.z, wb.w));
+                } else {
+                    *reinterpret_cast<uint2*>(cb) =
+                        make_uint2(e2m1x8(q0[0], q0[1], q0[2], q0[3], q0[4], q0[5], q0[6], q0[7]),
+                                   e2m1x8(q0[8], q0[9], q0[10], q0[11], q0[12], q0[13], q0[14], q0[15]));
+                    *reinterpret_cast<uint2*>(cb + ms2) =
+                        make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
+                                   e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
+                }
                 sb[0] = (uint8_t)sf0;
                 sb[ms16] = (uint8_t)sf1;
             }
@@ -757,7 +789,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
 }  // namespace
 
-template <bool RowRht>
+template <bool RowRht, bool SR>
 __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel(const __grid_constant__ NvParams p) {
     extern __shared__ __align__(1024) uint8_t nv_smem_raw[];
     uint8_t* const nv_smem = nv_smem_raw + ((1024u - (smem_u32(nv_smem_raw) & 1023u)) & 1023u);
@@ -805,7 +837,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
             mbar_wait_bounded(&sh.full[st], last_use & 1u, MBAR_LIMIT);
         }
     } else {
-        nv_consumer<RowRht>(p, sh, nv_smem, warp, lane);
+        nv_consumer<RowRht, SR>(p, sh, nv_smem, warp, lane);
     }
 
     // ---- the last CTA to leave publishes the section scales and resets the
@@ -845,12 +877,16 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
 
 int nvfp4_blocks_per_sm() {
     // both variants: the grid is sized for the one with fewer resident CTAs
-    int n0 = 0, n1 = 0;
-    cudaFuncSetAttribute(nvfp4_group_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
-    cudaFuncSetAttribute(nvfp4_group_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, nvfp4_group_kernel<false>, NV_THREADS, NV_DYN_SMEM);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, nvfp4_group_kernel<true>, NV_THREADS, NV_DYN_SMEM);
-    const int n = n0 < n1 ? n0 : n1;
+    // every variant: the grid is sized for the one with fewest resident CTAs
+    void (*const kernels[4])(NvParams) = {nvfp4_group_kernel<false, false>, nvfp4_group_kernel<true, false>,
+                                          nvfp4_group_kernel<false, true>, nvfp4_group_kernel<true, true>};
+    int n = 1 << 30;
+    for (auto* k : kernels) {
+        int m = 0;
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, k, NV_THREADS, NV_DYN_SMEM);
+        n = m < n ? m : n;
+    }
     return n > 0 ? n : 1;
 }
 
@@ -862,9 +898,13 @@ int nvfp4_tiles_in_flight_per_cta() { return NST + 2; }
 int nvfp4_tiles_per_claim() { return CLAIM; }
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
-    if (p.flags & HQ_ROW_RHT)
-        nvfp4_group_kernel<true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
-    else
-        nvfp4_group_kernel<false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+    const bool rot = p.flags & HQ_ROW_RHT, sr = p.flags & (HQ_ROW_SR | HQ_COL_SR);
+    if (sr) {
+        if (rot) nvfp4_group_kernel<true, true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+        else nvfp4_group_kernel<false, true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+    } else {
+        if (rot) nvfp4_group_kernel<true, false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+        else nvfp4_group_kernel<false, false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
+    }
 }
 }  // namespace hq

@@ -71,6 +71,21 @@ def test_group_rht_quant_argument_errors(L):
     assert _grp(L, flags=0) == hq.HQ_ERR_UNSUPPORTED
     assert _grp(L, flags=16) == hq.HQ_ERR_UNSUPPORTED
     assert _grp(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_RHT) == hq.HQ_ERR_UNSUPPORTED  # rotation without rows
+    assert _grp(L, flags=3 | hq.HQ_COL_SR) == hq.HQ_ERR_UNSUPPORTED               # needs the _sr entry (a seed)
+
+
+def _grp_sr(L, flags=3 | 32 | 64, offset=0, seed=7):
+    arr = (ctypes.c_int64 * 2)(128, 128)
+    return L.hq_group_rht_quant_sr(P(FAKE), 256, 256, ctypes.cast(arr, P), 2, 0x1234, flags, seed, offset,
+                                   P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                                   P(FAKE), 4096, None)
+
+
+def test_group_rht_quant_sr_argument_errors(L):
+    assert _grp_sr(L, offset=8) == hq.HQ_ERR_ALIGN                        # offset % 16
+    assert _grp_sr(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_SR) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_sr(L, flags=hq.HQ_ROWWISE | hq.HQ_COL_SR) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_sr(L, flags=3 | 128) == hq.HQ_ERR_UNSUPPORTED
     assert _grp(L, x=0) == hq.HQ_ERR_NULL
     assert _grp(L, ws=0) == hq.HQ_ERR_NULL
     assert _grp(L, ptrs=0) == hq.HQ_ERR_NULL

@@ -73,7 +73,7 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
 
 
 @pytest.mark.parametrize("name,per_elem", [("grouped_moe", 3.125), ("grouped_moe_amax_given", 3.125),
-                                           ("grouped_moe_row_rht", 3.125), ("dense_nvfp4", 3.125), ("dsa_indexer", 3.03125),
+                                           ("grouped_moe_row_rht", 3.125), ("grouped_moe_sr", 3.125), ("dense_nvfp4", 3.125), ("dsa_indexer", 3.03125),
                                            ("dsa_indexer_nvfp4", 2.59375),
                                            ("qmoe_bf16", 3.03125), ("qmoe_swiglu", 9.03125)])
 def test_algorithmic_bytes(name, per_elem):

@@ -282,6 +282,59 @@ def test_amax_given_grouped_moe_16384x7168(hq):
     _check(got, want, x, splits, mask, 3)
 
 
+def _run_sr(hq, x, splits, mask, flags, seed, offset):
+    M, K = x.shape
+    out, bufs = _guarded_outputs(hq, M, K, len(splits), flags)
+    ws = hq.new_workspace(len(splits))
+    hq.group_rht_quant(_bf16_dev(x), splits, mask, flags, ws=ws, out=out, seed=seed, offset=offset)
+    torch.cuda.synchronize()
+    for k, raw in bufs.items():
+        assert torch.all(raw[-GUARD:] == 0xA5), f"guard band of {k} overwritten"
+    assert torch.count_nonzero(ws).item() == 0
+    return {k: v.cpu().numpy() for k, v in out.items()}
+
+
+@pytest.mark.parametrize("flags", [3 | 32 | 64, 1 | 32, 2 | 64, 3 | 64, 1 | 4 | 32, 3 | 4 | 32 | 64 | 8])
+def test_stochastic_rounding_matches_oracle(hq, flags):
+    """Stochastic rounding is decided by integer comparisons of exact values,
+    so the codes must be bit-identical to the oracle's."""
+    splits = [128, 0, 256, 128]
+    x = _case(501, 384, splits)
+    mask, seed, offset = 0x6B2D, 0x0123456789ABCDEF, 16 * 12345
+    got = _run_sr(hq, x, splits, mask, flags, seed, offset)
+    base = flags & (1 | 2 | 4 | 32 | 64)
+    want = oracle.group_rht_quant(x, splits, mask, base, seed=seed, offset=offset)
+    for k in want:
+        assert_bits_equal(got[k], want[k], k)
+
+
+def test_stochastic_rounding_depends_only_on_seed_and_offset(hq):
+    splits = [256, 128]
+    x = _case(511, 256, splits)
+    a = _run_sr(hq, x, splits, 0x1111, 3 | 32 | 64, 5, 0)
+    b = _run_sr(hq, x, splits, 0x1111, 3 | 32 | 64 | 8, 5, 0)          # another schedule: same codes
+    c = _run_sr(hq, x, splits, 0x1111, 3 | 32 | 64, 6, 0)
+    d = _run_sr(hq, x, splits, 0x1111, 3 | 32 | 64, 5, 16)
+    for k in a:
+        assert_bits_equal(b[k], a[k], k)
+    for other in (c, d):
+        assert not np.array_equal(other["row_codes"], a["row_codes"])
+        assert not np.array_equal(other["col_codes"], a["col_codes"])
+        assert_bits_equal(other["row_sf"], a["row_sf"], "row_sf")
+
+
+@pytest.mark.slow
+def test_stochastic_rounding_grouped_moe_16384x7168(hq):
+    seed = S.SEEDS["grouped_moe"]
+    x = S.normal_bf16(seed, (16384, 7168))
+    splits = S.moe_splits(seed)
+    mask = S.sign_mask16(seed)
+    got = _run_sr(hq, x, splits, mask, 3 | 32 | 64, 2024, 1 << 20)
+    want = oracle.group_rht_quant(x, splits, mask, 3 | 32 | 64, seed=2024, offset=1 << 20)
+    for k in want:
+        assert_bits_equal(got[k], want[k], k)
+
+
 def test_bounded_wait_reports_timeout_and_recovers(hq):
     """A workspace outside its rest state makes the cast tiles' wait run out:
     one section of 4 column tiles is 4 amax tiles (items 0..3) then 4 cast
