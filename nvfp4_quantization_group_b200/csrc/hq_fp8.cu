@@ -334,11 +334,14 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
 // two consecutive groups (adjacent in memory) per step.  BF16 / FP32 input:
 // the raw load words of the next batch of steps are fetched before the
 // current batch is computed (two register buffers), so loads stay in flight
-// during the arithmetic.  SwiGLU input: compute-heavy, loads of a batch
-// first and then its arithmetic.
+// during the arithmetic; the same for the SwiGLU input (gate and up words).
 template <int MODE> struct K128Raw;
 template <> struct K128Raw<HQ_ACT_NONE_BF16> { static constexpr int U = 4; uint4 w[U]; };
 template <> struct K128Raw<HQ_ACT_NONE_F32> { static constexpr int U = 2; uint4 w[U][2]; };
+#ifndef HQ_K128_SWIGLU_U
+#define HQ_K128_SWIGLU_U 1  // steps per buffer (2 or more: register pressure halves the occupancy, 30 % slower)
+#endif
+template <> struct K128Raw<HQ_ACT_SWIGLU_F32> { static constexpr int U = HQ_K128_SWIGLU_U; uint4 w[U][4]; };
 
 // Scale, codes and the stores of one group whose negated values are ny
 // (AMAX: the group's amax too).
@@ -380,8 +383,9 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
     const uint32_t ngroups = (uint32_t)p.ngroups;  // < 2^31 (host check)
     const uint32_t npairs = (ngroups + 1) >> 1;
 
-    if constexpr (MODE != HQ_ACT_SWIGLU_F32) {
+    {
         using Raw = K128Raw<MODE>;
+        const uint32_t gpr = (uint32_t)(p.K_out / 128);  // groups per row (SwiGLU addressing)
         constexpr int U = Raw::U;
         const uint32_t stride = nwarps * U;
         auto load = [&](uint32_t base, Raw& r) {
@@ -392,6 +396,17 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
                 if constexpr (MODE == HQ_ACT_NONE_BF16) {
                     r.w[u] = ok ? ld_nc_v4(reinterpret_cast<const uint16_t*>(p.in) + (uint64_t)g * 128 + 8 * l)
                                 : make_uint4(0u, 0u, 0u, 0u);
+                } else if constexpr (MODE == HQ_ACT_SWIGLU_F32) {
+                    // gate = columns [0, K_out) of the row, up = [K_out, 2 K_out)
+                    uint32_t colg;
+                    const uint32_t row = udivmod(ok ? g : 0u, gpr, p.gpr_magic, colg);
+                    const float* gate = reinterpret_cast<const float*>(p.in) + (uint64_t)row * 2 * p.K_out + colg * 128;
+                    const float* up = gate + p.K_out;
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    r.w[u][0] = ok ? ld_nc_v4(gate + 4 * l) : z;
+                    r.w[u][1] = ok ? ld_nc_v4(gate + 64 + 4 * l) : z;
+                    r.w[u][2] = ok ? ld_nc_v4(up + 4 * l) : z;
+                    r.w[u][3] = ok ? ld_nc_v4(up + 64 + 4 * l) : z;
                 } else {
                     const float* in = reinterpret_cast<const float*>(p.in) + (uint64_t)g * 128;
                     r.w[u][0] = ok ? ld_nc_v4(in + 4 * l) : make_uint4(0u, 0u, 0u, 0u);
@@ -412,6 +427,15 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
                     ny[1] = bf16x2_to_f2(w.y ^ 0x80008000u);
                     ny[2] = bf16x2_to_f2(w.z ^ 0x80008000u);
                     ny[3] = bf16x2_to_f2(w.w ^ 0x80008000u);
+                } else if constexpr (MODE == HQ_ACT_SWIGLU_F32) {
+                    const uint4 g0 = r.w[u][0], g1 = r.w[u][1], u0 = r.w[u][2], u1 = r.w[u][3];
+                    const uint32_t gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    const uint32_t uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                    float act[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) act[j] = neg_swiglu(__uint_as_float(gg[j]), __uint_as_float(uu[j]));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) ny[j] = pack2(act[2 * j], act[2 * j + 1]);
                 } else {
                     const uint4 w0 = r.w[u][0], w1 = r.w[u][1];
                     ny[0] = pack2(-__uint_as_float(w0.x), -__uint_as_float(w0.y));
@@ -433,40 +457,6 @@ __global__ void __launch_bounds__(K128_THREADS) k128_fp8_kernel(K128Params p) {
             load(base + stride, r0);
             compute(base, r1);
             base += stride;
-        }
-    } else {
-        const uint32_t gpr = (uint32_t)(p.K_out / 128);  // groups per row
-        for (uint32_t base = warp * K128_UNROLL; base < npairs; base += nwarps * K128_UNROLL) {
-            f2 ny[K128_UNROLL][4];
-            // ---- loads and activation (all steps first)
-#pragma unroll
-            for (int u = 0; u < K128_UNROLL; ++u) {
-                const uint32_t g = (base + u) * 2 + half;
-                if (base + u < npairs && g < ngroups) {
-                    uint32_t colg;
-                    const uint32_t row = udivmod(g, gpr, p.gpr_magic, colg);
-                    const float* gate = reinterpret_cast<const float*>(p.in) + (uint64_t)row * 2 * p.K_out + colg * 128;
-                    const float* up = gate + p.K_out;
-                    uint4 g0 = ld_nc_v4(gate + 4 * l), g1 = ld_nc_v4(gate + 64 + 4 * l);
-                    uint4 u0 = ld_nc_v4(up + 4 * l), u1 = ld_nc_v4(up + 64 + 4 * l);
-                    const uint32_t gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                    const uint32_t uu[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-                    float act[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        act[j] = neg_swiglu(__uint_as_float(gg[j]), __uint_as_float(uu[j]));
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) ny[u][j] = pack2(act[2 * j], act[2 * j + 1]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) ny[u][j] = 0;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < K128_UNROLL; ++u) {
-                const uint32_t g = (base + u) * 2 + half;
-                k128_finish<AMAX>(p, g, base + u < npairs && g < ngroups, l, ny[u], true);
-            }
         }
     }
 }
