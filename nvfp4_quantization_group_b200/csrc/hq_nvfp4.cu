@@ -143,6 +143,42 @@ __device__ __forceinline__ void rht_stages(f2 (&v)[16]) {
     }
 }
 
+// max over the 16 outputs of the last butterfly stage (h = 8) of |v|, both
+// halves, and m, without forming the outputs: for the pair (a, b) the stage
+// writes RN(a + b) and RN(a - b), and the larger magnitude of the two is
+// RN(|a| + |b|) (the operation whose operands have equal signs adds the
+// magnitudes; the other one's magnitude is RN(||a| - |b||), no larger, as
+// rounding is monotone and symmetric).  NaN sums are skipped like NaN outputs.
+__device__ __forceinline__ float last_stage_absmax(const f2 (&v)[16], float m) {
+    float s[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float a0, a1, b0, b1;
+        unpack2(v[i], a0, a1);
+        unpack2(v[i + 8], b0, b1);
+        s[2 * i] = __fadd_rn(fabsf(a0), fabsf(b0));
+        s[2 * i + 1] = __fadd_rn(fabsf(a1), fabsf(b1));
+    }
+    const float p = max3(max3(s[0], s[1], s[2]), max3(s[3], s[4], s[5]), max3(s[6], s[7], s[8]));
+    const float q = max3(max3(s[9], s[10], s[11]), max3(s[12], s[13], s[14]), max3(s[15], m, 0.0f));
+    return max3(p, q, 0.0f);
+}
+
+// Butterfly stages 2 and 4 (the first three stages with stage 1).
+__device__ __forceinline__ void rht_stages_24(f2 (&v)[16]) {
+#pragma unroll
+    for (int h = 2; h < 8; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & h) == 0) {
+                const f2 a = v[i], b = v[i + h];
+                v[i] = add2(a, b);
+                v[i + h] = sub2(a, b);
+            }
+        }
+    }
+}
+
 // Unnormalised column RHT, H16 diag(sigma), of a BF16 column pair (16 rows):
 // two columns per packed f32x2 lane; stages 1, 2, 4, 8 in ascending order.
 __device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t (&sg)[16], f2 (&v)[16]) {
@@ -150,13 +186,22 @@ __device__ __forceinline__ void column_rht(const uint32_t (&w)[16], const bf16_t
     for (int i = 0; i < 16; i += 2) rht_stage1(w[i], w[i + 1], sg[i], sg[i + 1], v[i], v[i + 1]);
     rht_stages(v);
 }
+// max(m, |column RHT outputs|) of a BF16 column pair: stages 1, 2, 4 and the
+// last stage's maximum by last_stage_absmax.
+__device__ __forceinline__ float column_rht_absmax(const uint32_t (&w)[16], const bf16_t (&sg)[16], float m) {
+    f2 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) rht_stage1(w[i], w[i + 1], sg[i], sg[i + 1], v[i], v[i + 1]);
+    rht_stages_24(v);
+    return last_stage_absmax(v, m);
+}
 
 // Unnormalised RHT along K of one 16-column block of two rows a and b (word c
 // holds elements 2c, 2c + 1, the even one in the low half): v[i] = {a_i, b_i}
 // of the output.  Stage 1 pairs the two halves of a word, with the signs
 // folded in as in rht_stage1.
-__device__ __forceinline__ void row_rht(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const bf16_t (&sg)[16],
-                                        f2 (&v)[16]) {
+__device__ __forceinline__ void row_rht_stage1(const uint32_t (&wa)[8], const uint32_t (&wb)[8],
+                                               const bf16_t (&sg)[16], f2 (&v)[16]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         bf16_t a0, a1, b0, b1;
@@ -166,6 +211,10 @@ __device__ __forceinline__ void row_rht(const uint32_t (&wa)[8], const uint32_t 
         v[2 * c] = pack2(fma_bf16(a0, sg[2 * c], pa), fma_bf16(b0, sg[2 * c], pb));
         v[2 * c + 1] = pack2(fma_bf16(a0, sg[2 * c], -pa), fma_bf16(b0, sg[2 * c], -pb));
     }
+}
+__device__ __forceinline__ void row_rht(const uint32_t (&wa)[8], const uint32_t (&wb)[8], const bf16_t (&sg)[16],
+                                        f2 (&v)[16]) {
+    row_rht_stage1(wa, wb, sg, v);
     rht_stages(v);
 }
 
@@ -563,6 +612,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         q.rs_off0 = (uint64_t)rr * K16 + b;
         return q;
     };
+    Part parts[16 / NCW];  // the same for every tile
+#pragma unroll
+    for (int pi = 0; pi < 16 / NCW; ++pi) parts[pi] = part(w + pi * NCW);
 
     for (uint32_t k = 0;; ++k) {
         const int st = (int)(k % NST);
@@ -591,17 +643,14 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             float mrf = 0.0f, mcol = 0.0f;
 #pragma unroll
             for (int pi = 0; pi < 16 / NCW; ++pi) {
-            const int vw = w + pi * NCW;
-            const Part pt = part(vw);
+            const Part& pt = parts[pi];
             if (do_row && RowRht) {
                 uint32_t wa[8], wb[8];
                 load_row_pair(pt, wa, wb);
                 f2 v[16];
-                row_rht(wa, wb, sg, v);
-                float r0[16], r1[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) unpack2(v[i], r0[i], r1[i]);
-                mrf = max3(mrf, absmax16(r0), absmax16(r1));
+                row_rht_stage1(wa, wb, sg, v);
+                rht_stages_24(v);
+                mrf = last_stage_absmax(v, mrf);
             } else if (do_row) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
@@ -617,22 +666,15 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 uint32_t x[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) x[i] = *reinterpret_cast<const uint32_t*>(T + pt.coff + 1024 * i);
-                f2 v[16];
-                column_rht(x, sg, v);
-                float c0[16], c1[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) unpack2(v[i], c0[i], c1[i]);
-                mcol = max3(mcol, absmax16(c0), absmax16(c1));
+                mcol = column_rht_absmax(x, sg, mcol);
             }
             }  // parts
             // rotated rows: the maximum of |0.25 y| as binary32 bits (>= 0:
             // integer order)
             if (RowRht) mrow = __float_as_uint(__fmul_rn(mrf, 0.25f));
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                mrow = max(mrow, __shfl_xor_sync(0xFFFFFFFFu, mrow, o));
-                mcol = fmaxf(mcol, __shfl_xor_sync(0xFFFFFFFFu, mcol, o));
-            }
+            // (both non-negative and not NaN: binary32 bits order as integers)
+            mrow = __reduce_max_sync(0xFFFFFFFFu, mrow);
+            mcol = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mcol)));
             if (lane == 0) {
                 // max |0.25 y| == RN(0.25 max |y|): rounding is monotone
                 atomicMax(&sh.acc_row[st], mrow);
@@ -658,8 +700,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             uint8_t* const rs_base = p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
 #pragma unroll
             for (int pi = 0; pi < 16 / NCW; ++pi) {
-            const int vw = w + pi * NCW;
-            const Part pt = part(vw);
+            const Part& pt = parts[pi];
             if (do_row && RowRht) {
                 uint32_t wa[8], wb[8];
                 load_row_pair(pt, wa, wb);
