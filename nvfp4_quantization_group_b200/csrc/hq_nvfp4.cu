@@ -639,7 +639,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
         if (!(h.flags & H_CAST)) {
             // ===================================================== amax tile
-            uint32_t mrow = 0u;
+            uint32_t mrow = 0u, mrow2 = 0u;  // mrow2: BF16 pair of running magnitude maxima
             float mrf = 0.0f, mcol = 0.0f;
 #pragma unroll
             for (int pi = 0; pi < 16 / NCW; ++pi) {
@@ -652,15 +652,19 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 rht_stages_24(v);
                 mrf = last_stage_absmax(v, mrf);
             } else if (do_row) {
+                // rows rr and rr + 4 into the running pair (a NaN is skipped:
+                // the maximum returns the other operand, and the running pair
+                // starts at zero)
+                uint32_t m[2];
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const uint32_t ro = pt.roff0 + 4096u * kk;
                     const uint4 lo = *reinterpret_cast<const uint4*>(T + ro);  // (odd chunk if swap)
                     const uint4 hi = *reinterpret_cast<const uint4*>(T + (ro + pt.roff2));
-                    const uint32_t m = hmax_abs(hmax_abs(hmax_abs(lo.x, lo.y), hmax_abs(lo.z, lo.w)),
-                                                hmax_abs(hmax_abs(hi.x, hi.y), hmax_abs(hi.z, hi.w)));
-                    mrow = max(mrow, halves_max_bits(m));
+                    m[kk] = hmax_abs(hmax_abs(hmax_abs(lo.x, lo.y), hmax_abs(lo.z, lo.w)),
+                                     hmax_abs(hmax_abs(hi.x, hi.y), hmax_abs(hi.z, hi.w)));
                 }
+                mrow2 = hmax_abs(mrow2, hmax_abs(m[0], m[1]));
             }
             if (do_col) {
                 uint32_t x[16];
@@ -671,7 +675,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
             }  // parts
             // rotated rows: the maximum of |0.25 y| as binary32 bits (>= 0:
             // integer order)
-            if (RowRht) mrow = __float_as_uint(__fmul_rn(mrf, 0.25f));
+            mrow = RowRht ? __float_as_uint(__fmul_rn(mrf, 0.25f)) : halves_max_bits(mrow2);
             // (both non-negative and not NaN: binary32 bits order as integers)
             mrow = __reduce_max_sync(0xFFFFFFFFu, mrow);
             mcol = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mcol)));
