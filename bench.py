@@ -312,12 +312,34 @@ class GroupedNVFP4(Workload):
         self.ws = self.hq.new_workspace(len(self.splits))
         return self.hq.group_outputs(self.M, self.K, len(self.splits))
 
+    def flags(self):
+        hq = self.hq
+        return hq.HQ_ROWWISE | hq.HQ_COLWISE | (0 if self.schedule == "fused" else hq.HQ_TWO_PASS)
+
+    sr_seed = None          # stochastic rounding seed of the host-buffer call (None: nearest)
+    host_pipeline = True    # end to end through hq_group_rht_quant_host
+
     def call(self, inputs, out):
         hq = self.hq
-        flags = hq.HQ_ROWWISE | hq.HQ_COLWISE | (0 if self.schedule == "fused" else hq.HQ_TWO_PASS)
-        hq.hq_group_rht_quant(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask, flags,
+        hq.hq_group_rht_quant(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask, self.flags(),
                               out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
                               out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
+
+    # end to end: the host-buffer entry, which overlaps the copies in, the
+    # casts and the copies out by groups of whole sections
+    def setup_e2e(self, host):
+        if not self.host_pipeline:
+            return super().setup_e2e(host)
+        torch, hq = self.torch, self.hq
+        self.h_in = {"x": self._pinned(torch, host["x"])}
+        self.h_out = hq.host_outputs(self.M, self.K, len(self.splits), self.flags())
+        self.staging = hq.HostStaging(self.M, self.K, len(self.splits))
+
+    def e2e_step(self):
+        if not self.host_pipeline:
+            return super().e2e_step()
+        self.hq.group_rht_quant_host(self.h_in["x"], self.splits, self.mask, self.flags(), staging=self.staging,
+                                     out=self.h_out, seed=self.sr_seed)
 
     def oracle_sample(self, host, rows=512):
         import oracle
@@ -333,6 +355,7 @@ class GroupedAmaxGiven(GroupedNVFP4):
     (HQ_AMAX_GIVEN): one pass over x.  The amax values come from one ordinary
     call before the timed steps."""
     name = "grouped_moe_amax_given"
+    host_pipeline = False   # (its amax inputs stay on the device)
 
     def setup(self, hq, torch, host):
         super().setup(hq, torch, host)
@@ -373,12 +396,8 @@ class GroupedRowRHT(GroupedNVFP4):
         c["directions"] = "rowwise (RHT16 along K) + columnwise"
         return c
 
-    def call(self, inputs, out):
-        hq = self.hq
-        flags = hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_ROW_RHT | (0 if self.schedule == "fused" else hq.HQ_TWO_PASS)
-        hq.hq_group_rht_quant(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask, flags,
-                              out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
-                              out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
+    def flags(self):
+        return super().flags() | self.hq.HQ_ROW_RHT
 
     def oracle_sample(self, host, rows=512):
         import oracle
@@ -399,10 +418,16 @@ class GroupedSR(GroupedNVFP4):
         c["workload"] += ", stochastic rounding (rowwise and columnwise codes)"
         return c
 
+    sr_seed = 1234
+
+    def flags(self):
+        hq = self.hq
+        return hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_ROW_SR | hq.HQ_COL_SR
+
     def call(self, inputs, out):
         hq = self.hq
         hq.hq_group_rht_quant_sr(inputs["x"], self.M, self.K, self.splits, len(self.splits), self.mask,
-                                 hq.HQ_ROWWISE | hq.HQ_COLWISE | hq.HQ_ROW_SR | hq.HQ_COL_SR, 1234, 0,
+                                 self.flags(), self.sr_seed, 0,
                                  out["row_codes"], out["row_sf"], out["col_codes"], out["col_sf"],
                                  out["amax_row"], out["amax_col"], out["sdec_row"], out["sdec_col"], self.ws)
 

@@ -200,6 +200,46 @@ hq_status hq_group_rht_quant_sr(const void *x, int64_t M, int64_t K,
                                 void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The grouped cast with x and every output in HOST memory: the rows are
+ * copied to the device, cast and copied back in groups of whole sections, so
+ * the copies of one group overlap the cast of the next and the copies in the
+ * other direction (page-locked host buffers are needed for the overlap;
+ * pageable ones give the same results, copied without overlap).  The codes
+ * and scales are those of hq_group_rht_quant_sr on the whole tensor (without
+ * HQ_ROW_SR / HQ_COL_SR, those of hq_group_rht_quant); a section's amax never
+ * crosses groups, and the random byte streams keep their element indices.
+ *  x, row_codes, row_sf, col_codes, col_sf, amax_row, amax_col, sdec_row,
+ *  sdec_col      host buffers with the layouts of hq_group_rht_quant; with
+ *                HQ_AMAX_GIVEN amax_* are read (host) and copied in.
+ *  seed, offset  as hq_group_rht_quant_sr (ignored without the SR flags).
+ *  dev_buf, dev_buf_bytes  device staging memory, >=
+ *                hq_group_rht_quant_host_device_bytes(M, K, S), 256-byte
+ *                aligned; it holds x, the outputs and the workspace (kept in
+ *                its rest state by the calls; zero it once before the first).
+ *  groups        section groups (1..HQ_HOST_MAX_GROUPS); 0 picks 8.
+ *  stream        the cast runs here; the call is ordered after the work
+ *                already on it, and work enqueued on it afterwards runs after
+ *                the last copy back (synchronize it before reading outputs).
+ *  h2d_stream, d2h_stream  two further streams for the copies (distinct from
+ *                stream and from each other).
+ * A fixed set of CUDA events per device is created on the first call; calls
+ * from several host threads are serialized while they enqueue.
+ * Errors: as hq_group_rht_quant_sr, HQ_ERR_WORKSPACE when dev_buf is too
+ *         small, HQ_ERR_UNSUPPORTED for a bad group count or stream set.
+ */
+#define HQ_HOST_MAX_GROUPS 32
+size_t hq_group_rht_quant_host_device_bytes(int64_t M, int64_t K, int S);
+hq_status hq_group_rht_quant_host(const void *x, int64_t M, int64_t K,
+                                  const int64_t *split_rows, int S, uint16_t sign_mask,
+                                  unsigned flags, uint64_t seed, uint64_t offset,
+                                  uint8_t *row_codes, uint8_t *row_sf,
+                                  uint8_t *col_codes, uint8_t *col_sf,
+                                  float *amax_row, float *amax_col,
+                                  float *sdec_row, float *sdec_col,
+                                  void *dev_buf, size_t dev_buf_bytes, int groups,
+                                  void *stream, void *h2d_stream, void *d2h_stream);
+
+/*
  * hq_group_rht_quant without a caller workspace, for callers that cannot
  * allocate device memory where they quantize (code running while a CUDA
  * graph is captured, plugins whose host framework owns all device memory,

@@ -27,10 +27,12 @@ HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
 HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
 HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1
 HQ_MAX_SECTIONS = 256
+HQ_HOST_MAX_GROUPS = 32
 
 EXPORTED = (
     "hq_version", "hq_status_string", "hq_group_rht_quant_workspace_size", "hq_workspace_init",
-    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_sr", "hq_group_rht_quant_noalloc", "hq_cat_rotate_fp8",
+    "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_sr", "hq_group_rht_quant_noalloc",
+    "hq_group_rht_quant_host", "hq_group_rht_quant_host_device_bytes", "hq_cat_rotate_fp8",
     "hq_cat_rotate_fp8_workspace_size", "hq_cat_rotate_nvfp4", "hq_cat_rotate_nvfp4_workspace_size",
     "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
 )
@@ -73,6 +75,11 @@ def lib() -> ctypes.CDLL:
         L.hq_group_rht_quant_noalloc.restype = c_int
         L.hq_group_rht_quant_noalloc.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u,
                                                  P, P, P, P, P, P, P, P, P]
+        L.hq_group_rht_quant_host_device_bytes.restype = sz
+        L.hq_group_rht_quant_host_device_bytes.argtypes = [i64, i64, c_int]
+        L.hq_group_rht_quant_host.restype = c_int
+        L.hq_group_rht_quant_host.argtypes = [P, i64, i64, P, c_int, ctypes.c_uint16, u, ctypes.c_uint64,
+                                              ctypes.c_uint64, P, P, P, P, P, P, P, P, P, sz, c_int, P, P, P]
         L.hq_cat_rotate_fp8.restype = c_int
         L.hq_cat_rotate_fp8.argtypes = [P, i64, c_int, P, i64, c_int, i64, c_int, c_int,
                                         P, P, c_int, i64, P, P, sz, P]
@@ -111,6 +118,10 @@ def _stream(stream):
     if isinstance(stream, int):
         return ctypes.c_void_p(stream)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _stream_or_null(stream):
+    return None if stream is None else _stream(stream)
 
 
 def _check(status: int, what: str) -> None:
@@ -170,6 +181,25 @@ def hq_group_rht_quant_noalloc(x, M, K, split_rows, S, sign_mask, flags, row_cod
                                             _p(sdec_col), _stream(stream)), "hq_group_rht_quant_noalloc")
 
 
+def hq_group_rht_quant_host_device_bytes(M: int, K: int, S: int) -> int:
+    return int(lib().hq_group_rht_quant_host_device_bytes(int(M), int(K), int(S)))
+
+
+def hq_group_rht_quant_host(x, M, K, split_rows, S, sign_mask, flags, seed, offset, row_codes, row_sf, col_codes,
+                            col_sf, amax_row, amax_col, sdec_row, sdec_col, dev_buf, groups=0, stream=None,
+                            h2d_stream=None, d2h_stream=None) -> None:
+    """x and the outputs are CPU tensors (page-locked for overlap); dev_buf a CUDA byte tensor of at least
+    hq_group_rht_quant_host_device_bytes(M, K, S), zeroed once."""
+    splits = (ctypes.c_int64 * len(split_rows))(*[int(v) for v in split_rows])
+    _check(lib().hq_group_rht_quant_host(_p(x), int(M), int(K), ctypes.cast(splits, ctypes.c_void_p), int(S),
+                                         int(sign_mask) & 0xFFFF, int(flags), int(seed) & (2**64 - 1),
+                                         int(offset) & (2**64 - 1), _p(row_codes), _p(row_sf), _p(col_codes),
+                                         _p(col_sf), _p(amax_row), _p(amax_col), _p(sdec_row), _p(sdec_col),
+                                         _p(dev_buf), 0 if dev_buf is None else dev_buf.numel() * dev_buf.element_size(),
+                                         int(groups), _stream(stream), _stream_or_null(h2d_stream),
+                                         _stream_or_null(d2h_stream)), "hq_group_rht_quant_host")
+
+
 def hq_cat_rotate_fp8(a, a_row_stride, a_width, b, b_row_stride, b_width, M, G, hadamard_n, out_fp8, scales,
                       scale_layout, scale_ld, amax_opt=None, stream=None) -> None:
     _check(lib().hq_cat_rotate_fp8(_p(a), int(a_row_stride), int(a_width), _p(b), int(b_row_stride),
@@ -208,6 +238,52 @@ def hq_convert(fmt, inp, out, n, stream=None) -> None:
 
 
 # ------------------------------------------------- allocating conveniences
+class HostStaging:
+    """Device staging memory and the two copy streams of hq_group_rht_quant_host, for one shape; reusable."""
+
+    def __init__(self, M: int, K: int, S: int, device="cuda"):
+        nbytes = hq_group_rht_quant_host_device_bytes(M, K, S)
+        if nbytes == 0:
+            raise HQError(HQ_ERR_SHAPE, "HostStaging")
+        self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)  # workspace rest state included
+        self.h2d = torch.cuda.Stream(device=device)
+        self.d2h = torch.cuda.Stream(device=device)
+
+
+def host_outputs(M: int, K: int, S: int, flags: int = HQ_ROWWISE | HQ_COLWISE, pin: bool = True) -> dict:
+    """Page-locked CPU output tensors for group_rht_quant_host (same names and shapes as group_outputs)."""
+    out = {}
+    u8 = dict(dtype=torch.uint8, pin_memory=pin)
+    f32 = dict(dtype=torch.float32, pin_memory=pin)
+    if flags & HQ_ROWWISE:
+        out.update(row_codes=torch.empty((M, K // 2), **u8), row_sf=torch.empty((M, K // 16), **u8),
+                   amax_row=torch.empty(S, **f32), sdec_row=torch.empty(S, **f32))
+    if flags & HQ_COLWISE:
+        out.update(col_codes=torch.empty(M * K // 2, **u8), col_sf=torch.empty(M * K // 16, **u8),
+                   amax_col=torch.empty(S, **f32), sdec_col=torch.empty(S, **f32))
+    return out
+
+
+def group_rht_quant_host(x: torch.Tensor, split_rows, sign_mask: int, flags: int = HQ_ROWWISE | HQ_COLWISE,
+                         staging: HostStaging | None = None, out: dict | None = None, groups: int = 0,
+                         stream=None, seed: int | None = None, offset: int = 0) -> dict:
+    """The grouped cast of a CPU BF16 [M, K] tensor into CPU outputs (hq_group_rht_quant_host): copies and
+    casts overlap by section groups.  The outputs are complete once `stream` (default: the current one) is
+    synchronized."""
+    M, K = x.shape
+    S = len(split_rows)
+    if staging is None:
+        staging = HostStaging(M, K, S)
+    if out is None:
+        out = host_outputs(M, K, S, flags)
+    g = out.get
+    hq_group_rht_quant_host(x, M, K, split_rows, S, sign_mask, flags, 0 if seed is None else seed, offset,
+                            g("row_codes"), g("row_sf"), g("col_codes"), g("col_sf"), g("amax_row"),
+                            g("amax_col"), g("sdec_row"), g("sdec_col"), staging.buf, groups, stream,
+                            staging.h2d, staging.d2h)
+    return out
+
+
 def new_workspace(num_sections: int, device="cuda", stream=None) -> torch.Tensor:
     """A workspace for `num_sections` sections, put into its rest state once."""
     nbytes = hq_group_rht_quant_workspace_size(num_sections)

@@ -1,5 +1,6 @@
 // hq_api.cu -- the extern "C" entry points of include/hq.h: argument checks,
-// kernel parameter blocks, grid sizing and launches.  No allocation, no
+// kernel parameter blocks, grid sizing and launches.  No allocation (a fixed
+// set of CUDA events per device for the host-buffer entry, created once), no
 // synchronization (hq_get_error excepted), no environment reads.
 #include <cudaTypedefs.h>
 #include <string.h>
@@ -76,6 +77,56 @@ bool encode_x_map(CUtensorMap* map, const void* x, int64_t M, int64_t K) {
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Offsets (bytes, 256-aligned) of the host-buffer entry's device staging:
+// x, the four code / scale buffers, the four per-section arrays, workspace.
+struct StagingLayout {
+    size_t x, row_codes, row_sf, col_codes, col_sf, amax_row, amax_col, sdec_row, sdec_col, ws, total;
+};
+StagingLayout staging_layout(int64_t M, int64_t K, int S, size_t ws_bytes) {
+    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    const size_t e = (size_t)M * (size_t)K;
+    StagingLayout L;
+    size_t o = 0;
+    L.x = o;         o = up(o + 2 * e);
+    L.row_codes = o; o = up(o + e / 2);
+    L.row_sf = o;    o = up(o + e / 16);
+    L.col_codes = o; o = up(o + e / 2);
+    L.col_sf = o;    o = up(o + e / 16);
+    L.amax_row = o;  o = up(o + 4 * (size_t)S);
+    L.amax_col = o;  o = up(o + 4 * (size_t)S);
+    L.sdec_row = o;  o = up(o + 4 * (size_t)S);
+    L.sdec_col = o;  o = up(o + 4 * (size_t)S);
+    L.ws = o;        o = up(o + ws_bytes);
+    L.total = o;
+    return L;
+}
+
+// Events of the host-buffer entry, per device: created on first use; a
+// mutex serializes the enqueueing of calls (a stream wait takes the event's
+// latest record at the time of the wait, so a later call may re-record).
+struct HostEvents {
+    cudaEvent_t start = nullptr, end = nullptr, in[HQ_HOST_MAX_GROUPS] = {}, out[HQ_HOST_MAX_GROUPS] = {};
+    bool ok = false;
+    std::mutex mu;
+};
+HostEvents g_host_ev[kMaxDevices];
+std::once_flag g_host_ev_once[kMaxDevices];
+
+HostEvents* host_events() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::call_once(g_host_ev_once[dev], [dev] {
+        HostEvents& h = g_host_ev[dev];
+        bool ok = cudaEventCreateWithFlags(&h.start, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&h.end, cudaEventDisableTiming) == cudaSuccess;
+        for (int g = 0; g < HQ_HOST_MAX_GROUPS && ok; ++g)
+            ok = cudaEventCreateWithFlags(&h.in[g], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h.out[g], cudaEventDisableTiming) == cudaSuccess;
+        h.ok = ok;
+    });
+    return g_host_ev[dev].ok ? &g_host_ev[dev] : nullptr;
 }
 
 }  // namespace
@@ -282,6 +333,133 @@ hq_status hq_group_rht_quant_sr(const void* x, int64_t M, int64_t K, const int64
                                 size_t ws_bytes, void* stream) {
     return group_rht_quant(x, M, K, split_rows, S, sign_mask, flags, seed, offset, row_codes, row_sf, col_codes,
                            col_sf, amax_row, amax_col, sdec_row, sdec_col, ws, ws_bytes, stream);
+}
+
+size_t hq_group_rht_quant_host_device_bytes(int64_t M, int64_t K, int S) {
+    if (S < 1 || S > HQ_MAX_SECTIONS || M < 0 || K <= 0 || K % NV_TILE != 0) return 0;
+    if (M * K >= ((int64_t)1 << 40) || M >= ((int64_t)1 << 31)) return 0;
+    return staging_layout(M, K, S, hq_group_rht_quant_workspace_size(S)).total;
+}
+
+hq_status hq_group_rht_quant_host(const void* x, int64_t M, int64_t K, const int64_t* split_rows, int S,
+                                  uint16_t sign_mask, unsigned flags, uint64_t seed, uint64_t offset,
+                                  uint8_t* row_codes, uint8_t* row_sf, uint8_t* col_codes, uint8_t* col_sf,
+                                  float* amax_row, float* amax_col, float* sdec_row, float* sdec_col,
+                                  void* dev_buf, size_t dev_buf_bytes, int groups, void* stream,
+                                  void* h2d_stream, void* d2h_stream) {
+    // ---- checks of what the per-group calls cannot see (they check the rest
+    // again on the staging pointers)
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR))
+        return HQ_ERR_UNSUPPORTED;
+    const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
+    if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_ROW_RHT) && !do_row) return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_ROW_SR) && !do_row) return HQ_ERR_UNSUPPORTED;
+    if ((flags & HQ_COL_SR) && !do_col) return HQ_ERR_UNSUPPORTED;
+    if ((flags & (HQ_ROW_SR | HQ_COL_SR)) && offset % 16 != 0) return HQ_ERR_ALIGN;
+    if (!split_rows || !dev_buf) return HQ_ERR_NULL;
+    if (S < 1 || S > HQ_MAX_SECTIONS || M < 0 || K <= 0) return HQ_ERR_SHAPE;
+    if (K % NV_TILE != 0) return HQ_ERR_ALIGN;
+    if (M * K >= ((int64_t)1 << 40) || M >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
+    int64_t total = 0;
+    for (int s = 0; s < S; ++s) {
+        if (split_rows[s] < 0) return HQ_ERR_SHAPE;
+        if (split_rows[s] % NV_TILE != 0) return HQ_ERR_ALIGN;
+        total += split_rows[s];
+    }
+    if (total != M) return HQ_ERR_SHAPE;
+    if (M > 0 && !x) return HQ_ERR_NULL;
+    if (do_row && (!amax_row || !sdec_row || (M > 0 && (!row_codes || !row_sf)))) return HQ_ERR_NULL;
+    if (do_col && (!amax_col || !sdec_col || (M > 0 && (!col_codes || !col_sf)))) return HQ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return HQ_ERR_ALIGN;
+    const size_t ws_bytes = hq_group_rht_quant_workspace_size(S);
+    const StagingLayout L = staging_layout(M, K, S, ws_bytes);
+    if (dev_buf_bytes < L.total) return HQ_ERR_WORKSPACE;
+    if (groups == 0) groups = 8;
+    if (groups < 1 || groups > HQ_HOST_MAX_GROUPS) return HQ_ERR_UNSUPPORTED;
+    if (h2d_stream == d2h_stream || h2d_stream == stream || d2h_stream == stream) return HQ_ERR_UNSUPPORTED;
+    HostEvents* ev = host_events();
+    if (!ev) return HQ_ERR_CUDA;
+
+    // ---- section groups of about M / groups rows (whole sections)
+    int gs[HQ_HOST_MAX_GROUPS + 1];
+    int ng = 0;
+    gs[0] = 0;
+    const int64_t target = (M + groups - 1) / groups;
+    int64_t acc = 0;
+    for (int s = 0; s < S; ++s) {
+        acc += split_rows[s];
+        if (acc >= target && acc > 0 && ng + 1 < groups && s + 1 < S) {
+            gs[++ng] = s + 1;
+            acc = 0;
+        }
+    }
+    gs[++ng] = S;
+
+    uint8_t* const base = static_cast<uint8_t*>(dev_buf);
+    const uint8_t* const hx = static_cast<const uint8_t*>(x);
+    const cudaStream_t st = (cudaStream_t)stream, hs = (cudaStream_t)h2d_stream, ds = (cudaStream_t)d2h_stream;
+    const size_t fS = 4 * (size_t)S;
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    std::lock_guard<std::mutex> lock(ev->mu);
+    // the copies start after the work already on `stream`
+    if (!ok(cudaEventRecord(ev->start, st)) || !ok(cudaStreamWaitEvent(hs, ev->start, 0)) ||
+        !ok(cudaStreamWaitEvent(ds, ev->start, 0)))
+        return HQ_ERR_CUDA;
+    if (flags & HQ_AMAX_GIVEN) {
+        if (do_row && !ok(cudaMemcpyAsync(base + L.amax_row, amax_row, fS, cudaMemcpyHostToDevice, hs)))
+            return HQ_ERR_CUDA;
+        if (do_col && !ok(cudaMemcpyAsync(base + L.amax_col, amax_col, fS, cudaMemcpyHostToDevice, hs)))
+            return HQ_ERR_CUDA;
+    }
+    int64_t r0 = 0;
+    for (int g = 0; g < ng; ++g) {
+        const int sa = gs[g], sb = gs[g + 1];
+        int64_t rows = 0;
+        for (int s = sa; s < sb; ++s) rows += split_rows[s];
+        const size_t e0 = (size_t)r0 * (size_t)K, e = (size_t)rows * (size_t)K;
+        if (rows > 0 && !ok(cudaMemcpyAsync(base + L.x + 2 * e0, hx + 2 * e0, 2 * e, cudaMemcpyHostToDevice, hs)))
+            return HQ_ERR_CUDA;
+        if (!ok(cudaEventRecord(ev->in[g], hs)) || !ok(cudaStreamWaitEvent(st, ev->in[g], 0))) return HQ_ERR_CUDA;
+        // the group's sections as one call; the random streams keep their
+        // element indices (offset + first element of the group)
+        const hq_status r = group_rht_quant(
+            base + L.x + 2 * e0, rows, K, split_rows + sa, sb - sa, sign_mask, flags, seed,
+            (flags & (HQ_ROW_SR | HQ_COL_SR)) ? offset + e0 : 0, do_row ? base + L.row_codes + e0 / 2 : nullptr,
+            do_row ? base + L.row_sf + e0 / 16 : nullptr, do_col ? base + L.col_codes + e0 / 2 : nullptr,
+            do_col ? base + L.col_sf + e0 / 16 : nullptr,
+            do_row ? reinterpret_cast<float*>(base + L.amax_row) + sa : nullptr,
+            do_col ? reinterpret_cast<float*>(base + L.amax_col) + sa : nullptr,
+            do_row ? reinterpret_cast<float*>(base + L.sdec_row) + sa : nullptr,
+            do_col ? reinterpret_cast<float*>(base + L.sdec_col) + sa : nullptr, base + L.ws, ws_bytes, stream);
+        if (r != HQ_OK) return r;
+        if (!ok(cudaEventRecord(ev->out[g], st)) || !ok(cudaStreamWaitEvent(ds, ev->out[g], 0))) return HQ_ERR_CUDA;
+        if (rows > 0) {
+            if (do_row && (!ok(cudaMemcpyAsync(row_codes + e0 / 2, base + L.row_codes + e0 / 2, e / 2,
+                                               cudaMemcpyDeviceToHost, ds)) ||
+                           !ok(cudaMemcpyAsync(row_sf + e0 / 16, base + L.row_sf + e0 / 16, e / 16,
+                                               cudaMemcpyDeviceToHost, ds))))
+                return HQ_ERR_CUDA;
+            if (do_col && (!ok(cudaMemcpyAsync(col_codes + e0 / 2, base + L.col_codes + e0 / 2, e / 2,
+                                               cudaMemcpyDeviceToHost, ds)) ||
+                           !ok(cudaMemcpyAsync(col_sf + e0 / 16, base + L.col_sf + e0 / 16, e / 16,
+                                               cudaMemcpyDeviceToHost, ds))))
+                return HQ_ERR_CUDA;
+        }
+        r0 += rows;
+    }
+    // the per-section arrays after the last group
+    if (do_row && ((!(flags & HQ_AMAX_GIVEN) &&
+                    !ok(cudaMemcpyAsync(amax_row, base + L.amax_row, fS, cudaMemcpyDeviceToHost, ds))) ||
+                   !ok(cudaMemcpyAsync(sdec_row, base + L.sdec_row, fS, cudaMemcpyDeviceToHost, ds))))
+        return HQ_ERR_CUDA;
+    if (do_col && ((!(flags & HQ_AMAX_GIVEN) &&
+                    !ok(cudaMemcpyAsync(amax_col, base + L.amax_col, fS, cudaMemcpyDeviceToHost, ds))) ||
+                   !ok(cudaMemcpyAsync(sdec_col, base + L.sdec_col, fS, cudaMemcpyDeviceToHost, ds))))
+        return HQ_ERR_CUDA;
+    // work enqueued on `stream` afterwards runs after the last copy back
+    if (!ok(cudaEventRecord(ev->end, ds)) || !ok(cudaStreamWaitEvent(st, ev->end, 0))) return HQ_ERR_CUDA;
+    return HQ_OK;
 }
 
 size_t hq_cat_rotate_fp8_workspace_size(void) { return 0; }

@@ -99,6 +99,43 @@ def test_group_rht_quant_sr_argument_errors(L):
     assert _grp(L, row_codes=FAKE + 4) == hq.HQ_ERR_ALIGN
 
 
+def _grp_host(L, flags=3, M=256, K=256, splits=(128, 128), x=FAKE, ptrs=FAKE, dev=0x100000, dev_bytes=None,
+              groups=0, streams=(1, 2, 3), offset=0, split_ptr=True):
+    arr = (ctypes.c_int64 * len(splits))(*splits)
+    nbytes = hq.hq_group_rht_quant_host_device_bytes(M, K, len(splits)) if dev_bytes is None else dev_bytes
+    return L.hq_group_rht_quant_host(P(x), M, K, ctypes.cast(arr, P) if split_ptr else None, len(splits), 0x1234,
+                                     flags, 7, offset, P(ptrs), P(ptrs), P(ptrs), P(ptrs), P(ptrs), P(ptrs),
+                                     P(ptrs), P(ptrs), P(dev), nbytes, groups, P(streams[0]), P(streams[1]),
+                                     P(streams[2]))
+
+
+def test_group_rht_quant_host_sizes_and_argument_errors(L):
+    # staging: x + codes + scales of both directions + 4 section arrays + workspace, 256-byte pieces
+    n = hq.hq_group_rht_quant_host_device_bytes(256, 256, 2)
+    e = 256 * 256
+    assert n >= 2 * e + 2 * (e // 2 + e // 16) + hq.hq_group_rht_quant_workspace_size(2) and n % 256 == 0
+    assert hq.hq_group_rht_quant_host_device_bytes(256, 200, 2) == 0        # K % 128
+    assert hq.hq_group_rht_quant_host_device_bytes(256, 256, 0) == 0
+    assert hq.hq_group_rht_quant_host_device_bytes(-1, 256, 1) == 0
+    assert _grp_host(L, flags=0) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, flags=3 | 128) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_SR) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, flags=3 | hq.HQ_COL_SR, offset=8) == hq.HQ_ERR_ALIGN
+    assert _grp_host(L, split_ptr=False) == hq.HQ_ERR_NULL
+    assert _grp_host(L, dev=0) == hq.HQ_ERR_NULL
+    assert _grp_host(L, x=0) == hq.HQ_ERR_NULL
+    assert _grp_host(L, ptrs=0) == hq.HQ_ERR_NULL
+    assert _grp_host(L, K=200) == hq.HQ_ERR_ALIGN
+    assert _grp_host(L, splits=(128, 256)) == hq.HQ_ERR_SHAPE
+    assert _grp_host(L, splits=(64, 192)) == hq.HQ_ERR_ALIGN
+    assert _grp_host(L, dev=0x100000 + 16) == hq.HQ_ERR_ALIGN               # staging 256-byte aligned
+    assert _grp_host(L, dev_bytes=n - 1) == hq.HQ_ERR_WORKSPACE
+    assert _grp_host(L, groups=hq.HQ_HOST_MAX_GROUPS + 1) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, groups=-1) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, streams=(1, 2, 2)) == hq.HQ_ERR_UNSUPPORTED         # copy streams must differ
+    assert _grp_host(L, streams=(1, 1, 3)) == hq.HQ_ERR_UNSUPPORTED
+
+
 def test_cat_rotate_fp8_argument_errors(L):
     def call(a=FAKE, a_rs=64 * 64, aw=64, b=FAKE, b_rs=64 * 64, bw=64, M=16, G=64, hn=128, out=FAKE,
              sc=FAKE, layout=0, ld=16, amax=None):
