@@ -13,10 +13,14 @@ the C ABI with pinned host buffers and the copies inside the timed region.
 The other workloads of the path (dense NVFP4, DSA indexer FP8, QMoE K128 FP8
 of BF16 and of SwiGLU) are reported under "workloads".
 
-Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
-events on the launching stream, with the L2 flushed (a 256 MiB write) before
-every step outside the events; barrier + synchronize around the timed region;
-the step time is the max over ranks.  Under torchrun every rank quantizes its
+Timing: W untimed warm-up steps, then exactly K steps on the launching
+stream between CUDA events; barrier + synchronize around the timed region;
+the step time is the max over ranks.  Inputs larger than L2 run the K steps
+back to back (no step finds its inputs in L2).  Smaller inputs get an L2
+flush before every step, outside the events: a 256 MiB write, then a 256 MiB
+read of another buffer, so that the step starts with none of its inputs and
+no dirty line in L2 (with the write alone, up to 126 MB of the flush's own
+dirty lines would be written back inside the timed step).  Under torchrun every rank quantizes its
 own batch (independent problems, no collective on the data path: weak
 scaling); torch.distributed only carries the barrier and the max of the times.
 
@@ -647,11 +651,25 @@ def l2_bytes(torch) -> int:
     return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
 
 
+class L2Flush:
+    """Before a step: write a buffer larger than L2, then read another one, so
+    that L2 holds neither the step's inputs nor dirty lines to write back."""
+
+    def __init__(self, torch):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
 def time_device(torch, wl: Workload, steps: int, warmup: int, ranks: Ranks, flush, force_flush=False):
     """Per-step milliseconds and how L2 was handled.  Inputs larger than L2:
     the steps run back to back (a step finds none of its inputs in L2; its own
     outputs' write-back is part of its traffic).  Smaller inputs: a 256 MiB
-    write flushes L2 before every step, outside the timed events."""
+    write and a 256 MiB read flush L2 before every step, outside the timed
+    events."""
     stream = torch.cuda.current_stream()
     l2 = l2_bytes(torch)
     if wl.input_bytes() > l2 and not force_flush:
@@ -673,21 +691,22 @@ def time_device(torch, wl: Workload, steps: int, warmup: int, ranks: Ranks, flus
                 "no flush")
         return [a.elapsed_time(b) / steps] * steps, note
     for _ in range(warmup):
-        flush.zero_()
+        flush()
         wl.step()
     torch.cuda.synchronize()
     ranks.barrier()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in evs:
-        flush.zero_()                      # L2 flush, outside the timed events
+        flush()                            # L2 flush, outside the timed events
         a.record(stream)
         wl.step()
         b.record(stream)
     torch.cuda.synchronize()
     ranks.barrier()
     torch.cuda.synchronize()
-    return [a.elapsed_time(b) for a, b in evs], f"flushed before every step ({L2_FLUSH_BYTES >> 20} MiB write)"
+    return [a.elapsed_time(b) for a, b in evs], (f"flushed before every step ({L2_FLUSH_BYTES >> 20} MiB write, then "
+                                                 f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)")
 
 
 def time_e2e(torch, wl: Workload, steps: int, warmup: int, ranks: Ranks) -> list:
@@ -784,7 +803,7 @@ def run_ours(args, ranks: Ranks) -> None:
     torch.cuda.set_device(ranks.local)
     ranks.init("nccl")
     peaks = measured_peaks()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch)
     gpu_index = torch.cuda.current_device()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -819,7 +838,7 @@ def run_ours(args, ranks: Ranks) -> None:
     if "ms_flushed" in main:
         line["l2_flushed"] = {"ms_per_step": round(main["ms_flushed"], 5),
                               "value": round(gbs(wl.alg_bytes() * world, main["ms_flushed"]), 2),
-                              "note": "the same steps with a 256 MiB write before each (outside the events)"}
+                              "note": "the same steps with the L2 flush before each (outside the events)"}
     if "e2e_ms" in main:
         line["e2e"] = {"value": round(gbs(wl.alg_bytes() * world, main["e2e_ms"]), 3), "unit": UNIT,
                        "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": wl.d2h_bytes(),

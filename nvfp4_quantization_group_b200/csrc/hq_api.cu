@@ -375,7 +375,7 @@ hq_status hq_group_rht_quant_host(const void* x, int64_t M, int64_t K, const int
     const size_t ws_bytes = hq_group_rht_quant_workspace_size(S);
     const StagingLayout L = staging_layout(M, K, S, ws_bytes);
     if (dev_buf_bytes < L.total) return HQ_ERR_WORKSPACE;
-    if (groups == 0) groups = 8;
+    if (groups == 0) groups = 16;
     if (groups < 1 || groups > HQ_HOST_MAX_GROUPS) return HQ_ERR_UNSUPPORTED;
     if (h2d_stream == d2h_stream || h2d_stream == stream || d2h_stream == stream) return HQ_ERR_UNSUPPORTED;
     HostEvents* ev = host_events();
