@@ -363,6 +363,15 @@ size_t hq_swiglu_fp8_k128_workspace_size(void);
  */
 hq_status hq_convert(int fmt, const float *in, uint8_t *out, int64_t n, void *stream);
 
+/*
+ * Element-wise stochastic E2M1 conversion with the device routine of
+ * hq_group_rht_quant_sr: out[i] (low nibble) is the code of in[i] rounded
+ * with random byte rnd[i] by that call's rule (|v| up to the next E2M1 value
+ * iff rnd[i] < floor(256 f); |v| >= 6 saturates; sign kept).  n >= 0; any
+ * alignment.  Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_CUDA.
+ */
+hq_status hq_convert_e2m1_sr(const float *in, const uint8_t *rnd, uint8_t *out, int64_t n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

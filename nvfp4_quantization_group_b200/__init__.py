@@ -34,7 +34,7 @@ EXPORTED = (
     "hq_get_error", "hq_group_rht_quant", "hq_group_rht_quant_sr", "hq_group_rht_quant_noalloc",
     "hq_group_rht_quant_host", "hq_group_rht_quant_host_device_bytes", "hq_cat_rotate_fp8",
     "hq_cat_rotate_fp8_workspace_size", "hq_cat_rotate_nvfp4", "hq_cat_rotate_nvfp4_workspace_size",
-    "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert",
+    "hq_swiglu_fp8_k128", "hq_swiglu_fp8_k128_workspace_size", "hq_convert", "hq_convert_e2m1_sr",
 )
 
 
@@ -96,6 +96,8 @@ def lib() -> ctypes.CDLL:
         L.hq_swiglu_fp8_k128_workspace_size.argtypes = []
         L.hq_convert.restype = c_int
         L.hq_convert.argtypes = [c_int, P, P, i64, P]
+        L.hq_convert_e2m1_sr.restype = c_int
+        L.hq_convert_e2m1_sr.argtypes = [P, P, P, i64, P]
         _lib = L
     return _lib
 
@@ -235,6 +237,10 @@ def hq_swiglu_fp8_k128_workspace_size() -> int:
 
 def hq_convert(fmt, inp, out, n, stream=None) -> None:
     _check(lib().hq_convert(int(fmt), _p(inp), _p(out), int(n), _stream(stream)), "hq_convert")
+
+
+def hq_convert_e2m1_sr(inp, rnd, out, n, stream=None) -> None:
+    _check(lib().hq_convert_e2m1_sr(_p(inp), _p(rnd), _p(out), int(n), _stream(stream)), "hq_convert_e2m1_sr")
 
 
 # ------------------------------------------------- allocating conveniences

@@ -582,4 +582,16 @@ hq_status hq_convert(int fmt, const float* in, uint8_t* out, int64_t n, void* st
     return launch_status();
 }
 
+hq_status hq_convert_e2m1_sr(const float* in, const uint8_t* rnd, uint8_t* out, int64_t n, void* stream) {
+    if (n < 0) return HQ_ERR_SHAPE;
+    if (n == 0) return HQ_OK;
+    if (!in || !rnd || !out) return HQ_ERR_NULL;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return HQ_ERR_CUDA;
+    const int64_t blocks = ((n + 3) / 4 + 255) / 256;
+    const int64_t cap = (int64_t)dev->sms * 16;
+    launch_convert_e2m1_sr(in, rnd, out, n, (int)(blocks < cap ? blocks : cap), (cudaStream_t)stream);
+    return launch_status();
+}
+
 }  // extern "C"

@@ -468,6 +468,27 @@ __global__ void convert_kernel(int fmt, const float* in, uint8_t* out, int64_t n
         out[i] = fmt == HQ_FMT_E4M3 ? e4m3_one(in[i]) : e2m1_one(in[i]);
 }
 
+// Four elements per thread: their random bytes packed as in the grouped
+// kernel (byte k for element k), one stochastic conversion of the four.
+__global__ void convert_e2m1_sr_kernel(const float* in, const uint8_t* rnd, uint8_t* out, int64_t n) {
+    const int64_t quads = (n + 3) / 4;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < quads;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        float v[4];
+        uint32_t w = 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int64_t i = 4 * q + k;
+            v[k] = i < n ? in[i] : 0.0f;
+            w |= (i < n ? (uint32_t)rnd[i] : 0u) << (8 * k);
+        }
+        const uint32_t c = e2m1x4_sr(v[0], v[1], v[2], v[3], w);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (4 * q + k < n) out[4 * q + k] = (uint8_t)((c >> (4 * k)) & 0xFu);
+    }
+}
+
 // ------------------------------------------------------------ launchers
 int cat_rotate_group_tiles(int G) { return (G + CAT_TG - 1) / CAT_TG; }
 
@@ -511,6 +532,11 @@ void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st) {
 
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st) {
     convert_kernel<<<grid, 256, 0, st>>>(fmt, in, out, n);
+}
+
+void launch_convert_e2m1_sr(const float* in, const uint8_t* rnd, uint8_t* out, int64_t n, int grid,
+                            cudaStream_t st) {
+    convert_e2m1_sr_kernel<<<grid, 256, 0, st>>>(in, rnd, out, n);
 }
 
 }  // namespace hq

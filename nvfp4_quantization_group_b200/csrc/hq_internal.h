@@ -52,6 +52,8 @@ int cat_rotate_group_tiles(int G);  // group tiles of the transposed-scale layou
 void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st, bool fp4);
 void launch_k128(int mode, const K128Params& p, int grid, cudaStream_t st);
 void launch_convert(int fmt, const float* in, uint8_t* out, int64_t n, int grid, cudaStream_t st);
+void launch_convert_e2m1_sr(const float* in, const uint8_t* rnd, uint8_t* out, int64_t n, int grid,
+                            cudaStream_t st);
 
 // exp(x) in binary32 by one fixed sequence of IEEE operations: Cody & Waite
 // reduction k = rint(x * log2(e)), r = (x - k*LN2_HI) - k*LN2_LO (two FMAs),

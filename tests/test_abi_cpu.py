@@ -193,6 +193,10 @@ def test_convert_and_workspace_argument_errors(L):
     assert L.hq_convert(0, P(FAKE), P(FAKE), -1, None) == hq.HQ_ERR_SHAPE
     assert L.hq_convert(0, P(FAKE), P(FAKE), 0, None) == hq.HQ_OK
     assert L.hq_convert(0, None, P(FAKE), 10, None) == hq.HQ_ERR_NULL
+    assert L.hq_convert_e2m1_sr(P(FAKE), P(FAKE), P(FAKE), -1, None) == hq.HQ_ERR_SHAPE
+    assert L.hq_convert_e2m1_sr(P(FAKE), P(FAKE), P(FAKE), 0, None) == hq.HQ_OK
+    assert L.hq_convert_e2m1_sr(P(FAKE), None, P(FAKE), 10, None) == hq.HQ_ERR_NULL
+    assert L.hq_convert_e2m1_sr(None, P(FAKE), P(FAKE), 10, None) == hq.HQ_ERR_NULL
     assert L.hq_workspace_init(None, 256, None) == hq.HQ_ERR_NULL
     assert L.hq_workspace_init(P(FAKE + 4), 256, None) == hq.HQ_ERR_ALIGN
     err = ctypes.c_uint32(0)

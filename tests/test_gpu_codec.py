@@ -51,6 +51,39 @@ def test_e4m3_conversion_matches_oracle(hq):
     assert np.all((nan & 0x7F) == 0x7F)
 
 
+def test_stochastic_e2m1_conversion_matches_oracle(hq):
+    """The device's stochastic E2M1 routine (the one hq_group_rht_quant_sr
+    uses) against the oracle's rule, element by element: a sweep of binary32
+    patterns over and around the E2M1 range with seeded random bytes, every
+    byte value for grid points, midpoints and values whose fraction is r/256
+    exactly or just above it, both zeros, saturation and infinities, and a
+    length that leaves a ragged group of four."""
+    rng = np.random.default_rng(77)
+    x = _bits_sweep(-8, 3, 17)
+    r = rng.integers(0, 256, size=x.size, dtype=np.uint8)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float32)
+    steps = np.array([0.5, 0.5, 0.5, 0.5, 1.0, 1.0, 2.0], dtype=np.float32)
+    special = [0.0, -0.0, 6.0, -6.0, 6.5, 7.0, 1e30, -1e30, np.inf, -np.inf, 5.999999, 1e-40, -1e-40]
+    for g, st in zip(grid[:-1], steps):
+        for f in (0, 1, 127, 128, 129, 254, 255):
+            v = np.float32(g + st * f / 256.0)
+            special += [v, -v, np.nextafter(v, np.float32(np.inf)), -np.nextafter(v, np.float32(np.inf))]
+    sp = np.array(special, dtype=np.float32)
+    xs = np.repeat(sp, 256)
+    rs = np.tile(np.arange(256, dtype=np.uint8), sp.size)
+    x = np.concatenate([x, xs, np.array([1.3, -2.6, 4.9], dtype=np.float32)])
+    r = np.concatenate([r, rs, np.array([7, 200, 99], dtype=np.uint8)])
+    assert x.size % 4 != 0
+    xd, rd = torch.from_numpy(x).cuda(), torch.from_numpy(r).cuda()
+    out = torch.empty(x.size, dtype=torch.uint8, device="cuda")
+    hq.hq_convert_e2m1_sr(xd, rd, out, x.size)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    want = oracle.e2m1_sr(x, r).astype(np.uint8)
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, (bad[:8], x[bad[:8]], r[bad[:8]], got[bad[:8]], want[bad[:8]])
+
+
 def test_e2m1_conversion_matches_oracle(hq):
     x = _bits_sweep(-5, 4, 3)
     x = np.concatenate([x, np.array([0.0, -0.0, 6.0, 7.0, 1e30, -1e30, 5.0, -5.0], dtype=np.float32)])
