@@ -222,10 +222,14 @@ hq_status hq_group_rht_quant_sr(const void *x, int64_t M, int64_t K,
  *                the last copy back (synchronize it before reading outputs).
  *  h2d_stream, d2h_stream  two further streams for the copies (distinct from
  *                stream and from each other).
- * A fixed set of CUDA events per device is created on the first call; calls
- * from several host threads are serialized while they enqueue.
+ * A fixed set of CUDA events per device is created on the first call and
+ * kept for the life of the process; calls from several host threads are
+ * serialized while they enqueue.
  * Errors: as hq_group_rht_quant_sr, HQ_ERR_WORKSPACE when dev_buf is too
  *         small, HQ_ERR_UNSUPPORTED for a bad group count or stream set.
+ *         Argument errors are found before anything is enqueued; a CUDA
+ *         error after the first group was enqueued returns HQ_ERR_CUDA with
+ *         the earlier groups' copies and casts still in flight.
  */
 #define HQ_HOST_MAX_GROUPS 32
 size_t hq_group_rht_quant_host_device_bytes(int64_t M, int64_t K, int S);
