@@ -129,17 +129,39 @@ __device__ __forceinline__ CatVec cat_vector(const CatRotateParams& p, uint32_t 
     return r;
 }
 
+// Where thread j's 16 elements of every vector come from in the wide layout
+// (whole segments in a or in b): the same input for all vectors, so the
+// choice and its strides are made once per thread.
+struct CatSrc {
+    const uint16_t* base;  // element 16j of vector (0, 0)
+    int64_t tstride;       // per row t
+    int gwidth;            // per group g
+};
+__device__ __forceinline__ CatSrc cat_src(const CatRotateParams& p, int j) {
+    const int a_chunks = p.a_width / 8;
+    CatSrc s;
+    if (2 * j < a_chunks) {
+        s.base = p.a + j * 16;
+        s.tstride = p.a_row_stride;
+        s.gwidth = p.a_width;
+    } else {
+        s.base = p.b + (2 * j - a_chunks) * 8;
+        s.tstride = p.b_row_stride;
+        s.gwidth = p.b_width;
+    }
+    return s;
+}
+
 // The two 16-byte chunks (elements 16j..16j+15) of vector (t, g).
-__device__ __forceinline__ void cat_load(const CatRotateParams& p, CatVec cv, int j, uint4& c0, uint4& c1) {
+__device__ __forceinline__ void cat_load(const CatRotateParams& p, const CatSrc& src, CatVec cv, int j, uint4& c0,
+                                         uint4& c1) {
     c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
     if (cv.t < 0) return;
     const int64_t t = cv.t;
     const int g = cv.g;
     const int a_chunks = p.a_width / 8;
     if (p.wide) {
-        const uint16_t* src = 2 * j < a_chunks ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + j * 16
-                                               : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (2 * j - a_chunks) * 8;
-        ld_nc_v8(src, c0, c1);
+        ld_nc_v8(src.base + (t * src.tstride + (int64_t)g * src.gwidth), c0, c1);
         return;
     }
 #pragma unroll
@@ -172,14 +194,15 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
     uint32_t tile = blockIdx.x;
     const uint32_t ntiles = (uint32_t)p.ntiles;
     uint4 n0, n1;  // the next tile's chunks
+    const CatSrc src = cat_src(p, j);
     CatVec nv = tile < ntiles ? cat_vector(p, tile, k) : none;
-    cat_load(p, nv, j, n0, n1);
+    cat_load(p, src, nv, j, n0, n1);
     for (; tile < ntiles; tile += gridDim.x) {
         const CatVec cv = nv;
         const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
         const uint32_t nt = tile + gridDim.x;
         nv = nt < ntiles ? cat_vector(p, nt, k) : none;
-        cat_load(p, nv, j, n0, n1);
+        cat_load(p, src, nv, j, n0, n1);
 
         // ---- elements 16j..16j+15 as 8 pairs (2i, 2i+1) of this segment
         f2 y[8];
