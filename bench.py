@@ -767,7 +767,10 @@ def run_reference(args, ranks: Ranks) -> None:
     line = {"impl": "reference", "metric": METRIC if wl.name == "grouped_moe" else f"{wl.name} GB/s",
             "value": round(v, 4), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic", "config": wl.config(),
+            "dtype": "f32", "data": "synthetic",
+            "config": dict(wl.config(), l2="host cores (the oracle)",
+                           parallelism=f"{args.gpus} independent batch(es), rank 0 times the oracle",
+                           alg_bytes_per_step_per_gpu=wl.alg_bytes(), elements_per_step_per_gpu=wl.elements()),
             "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{desc}; {nbytes} algorithmic bytes per step"},
             "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
