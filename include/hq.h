@@ -216,7 +216,10 @@ hq_status hq_group_rht_quant_sr(const void *x, int64_t M, int64_t K,
  *                hq_group_rht_quant_host_device_bytes(M, K, S), 256-byte
  *                aligned; it holds x, the outputs and the workspace (kept in
  *                its rest state by the calls; zero it once before the first).
- *  groups        section groups (1..HQ_HOST_MAX_GROUPS); 0 picks 16.
+ *  groups        section groups (1..HQ_HOST_MAX_GROUPS); 0 picks 16.  Groups
+ *                are cut at section boundaries only (a section's amax needs
+ *                all its rows), so S sections give at most S groups and a
+ *                single section is copied, cast and copied back in sequence.
  *  stream        the cast runs here; the call is ordered after the work
  *                already on it, and work enqueued on it afterwards runs after
  *                the last copy back (synchronize it before reading outputs).
