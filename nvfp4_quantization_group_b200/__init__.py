@@ -278,6 +278,8 @@ def group_rht_quant_host(x: torch.Tensor, split_rows, sign_mask: int, flags: int
     synchronized."""
     M, K = x.shape
     S = len(split_rows)
+    if (flags & (HQ_ROW_SR | HQ_COL_SR)) and seed is None:
+        raise HQError(HQ_ERR_UNSUPPORTED, "group_rht_quant_host: stochastic rounding needs a seed")
     if staging is None:
         staging = HostStaging(M, K, S)
     if out is None:

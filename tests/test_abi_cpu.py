@@ -136,6 +136,13 @@ def test_group_rht_quant_host_sizes_and_argument_errors(L):
     assert _grp_host(L, streams=(1, 1, 3)) == hq.HQ_ERR_UNSUPPORTED
 
 
+def test_host_wrapper_needs_a_seed_for_stochastic_rounding():
+    import torch
+    x = torch.zeros((128, 128), dtype=torch.bfloat16)
+    with pytest.raises(hq.HQError):
+        hq.group_rht_quant_host(x, [128], 0x1234, hq.HQ_ROWWISE | hq.HQ_ROW_SR)
+
+
 def test_cat_rotate_fp8_argument_errors(L):
     def call(a=FAKE, a_rs=64 * 64, aw=64, b=FAKE, b_rs=64 * 64, bw=64, M=16, G=64, hn=128, out=FAKE,
              sc=FAKE, layout=0, ld=16, amax=None):
