@@ -25,21 +25,28 @@ static_assert(((4 * (hq::NV_WS_HEADER + 3 * HQ_MAX_SECTIONS) + 255) & ~255) <= 3
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoallocWords];
 
 constexpr int kMaxDevices = 64;
-uint32_t* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+uint32_t* g_scratch_ptr[kMaxDevices];  // published only after a successful lookup
+std::mutex g_scratch_mu;
 
 // Device address of the scratch array on the current device.  In host code
 // the symbol is only a host-side stand-in, so the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, with that device current.  A successful lookup is
+// kept for the device; a failed one (e.g. made during a stream capture) is
+// not cached, so a later call tries again, and its error is cleared from the
+// runtime so that it is not reported by an unrelated later call.
 uint32_t* scratch_on_current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::call_once(g_scratch_once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        g_scratch_ptr[dev] = g_scratch_err[dev] == cudaSuccess ? static_cast<uint32_t*>(p) : nullptr;
-    });
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) {
+            g_scratch_ptr[dev] = static_cast<uint32_t*>(p);
+        } else {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+    }
     return g_scratch_ptr[dev];
 }
 
