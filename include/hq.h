@@ -259,7 +259,8 @@ hq_status hq_group_rht_quant_host(const void *x, int64_t M, int64_t K,
  * process exits.  The call allocates nothing: it clears the array with an
  * enqueued memset and launches the kernel.  The first call on a device looks
  * up the array's device address (cudaGetSymbolAddress) and so should come
- * before any stream capture.  All calls on a device share the one array:
+ * before any stream capture; a lookup that fails returns HQ_ERR_CUDA and is
+ * tried again by the next call.  All calls on a device share the one array:
  * calls that overlap on the GPU (different streams without ordering) race
  * and give wrong results.  A bounded device wait that gives up is not
  * reported by this entry point (there is no workspace to read it from).
