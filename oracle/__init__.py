@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             L.hqo_philox4x32_10.restype = None
             L.hqo_e2m1_sr_array.argtypes = [P, P, P, i64]
             L.hqo_e2m1_sr_array.restype = None
+            L.hqo_sf_swizzled_offset.argtypes = [i64, i64, i64]
+            L.hqo_sf_swizzled_offset.restype = i64
             _lib = L
     return _lib
 
@@ -130,6 +132,15 @@ def fwht(v: np.ndarray) -> np.ndarray:
 
 # -------------------------------------------------------------- operations
 ROWMAJOR, TRANSPOSED = 0, 1
+# scale formats: UE8M0 (power-of-two) FP8 scales, added to scale_layout / mode
+# of the FP8 calls; interleaved 128 x 4 NVFP4 block-scale tiles, added to the
+# grouped cast's flags and to the FP4 DSA call's scale_layout
+UE8M0, SF_SWIZZLED = 256, 128
+
+
+def sf_swizzled_offset(r: int, c: int, cols: int) -> int:
+    """Byte of element (r, c) of a [rows, cols] block-scale matrix in the interleaved tiles."""
+    return int(lib().hqo_sf_swizzled_offset(r, c, cols))
 
 
 def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=None,
@@ -150,7 +161,7 @@ def cat_rotate_fp8(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride=N
     else:
         b_w, b_rs = 0, 0
     out = np.empty((M, G * 128), dtype=np.uint8)
-    if scale_layout == ROWMAJOR:
+    if (scale_layout & 1) == ROWMAJOR:
         scales = np.empty((M, G), dtype=np.float32)
         ld = G
     else:
@@ -183,7 +194,7 @@ def cat_rotate_nvfp4(a, b, M, G, hadamard_n=128, a_row_stride=None, b_row_stride
     else:
         b_w, b_rs = 0, 0
     r = {"codes": np.empty((M, G * 64), dtype=np.uint8), "block_sf": np.empty((M, G * 8), dtype=np.uint8)}
-    if scale_layout == ROWMAJOR:
+    if (scale_layout & 1) == ROWMAJOR:
         r["sdec"] = np.empty((M, G), dtype=np.float32)
         ld = G
     else:
@@ -212,7 +223,7 @@ def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False, want_amax=False):
     the groups' amax [M, K_out/128]."""
     x = np.ascontiguousarray(x)
     out = np.empty((M, K_out), dtype=np.uint8)
-    scales = np.empty((M, K_out // 128), dtype=np.float32)
+    scales = np.empty((M, K_out // 128), dtype=np.float32)  # (mode may add UE8M0)
     pre = np.empty((M, K_out), dtype=np.float32) if want_pre else None
     amax = np.empty_like(scales) if want_amax else None
     rc = lib().hqo_swiglu_fp8_k128(mode, _ptr(x), M, K_out, _ptr(out), _ptr(scales), _ptr(amax), _ptr(pre))
@@ -221,7 +232,7 @@ def swiglu_fp8_k128(mode, x, M, K_out, want_pre=False, want_amax=False):
     return (out, scales, pre, amax) if want_amax else (out, scales, pre)
 
 
-ROWWISE, COLWISE, ROW_RHT, AMAX_GIVEN, ROW_SR, COL_SR = 1, 2, 4, 16, 32, 64
+ROWWISE, COLWISE, ROW_RHT, AMAX_GIVEN, ROW_SR, COL_SR = 1, 2, 4, 16, 32, 64  # (+ SF_SWIZZLED)
 
 
 def e2m1_sr(t, r):

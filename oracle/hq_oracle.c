@@ -38,6 +38,11 @@
  * the printed rule with exact rational quotients and crafted midpoint cases;
  * exp against FP64; NVFP4 against exact block-scale/code brute force,
  * dequantization bounds and the inverse-rotation round trip.
+ * Scale formats for direct GEMM consumption (TensorRT-LLM PR #15158 review
+ * thread: a use_ue8m0 option of the 1x128 quantizer; DeepGEMM issue #320: the
+ * tcgen05 data-path layouts of scale factors): UE8M0 FP8 scales and the
+ * 128 x 4 interleaved NVFP4 block-scale tiles, pinned by closed forms and an
+ * independent construction of the tile permutation.
  * Parity unpinned (readings the pages leave open, each moving results only
  * inside the 2^-20 midpoint window or the 1e-5 rotation tolerance): the
  * ascending butterfly stage order, and the operation order of the NVFP4
@@ -178,6 +183,45 @@ static float c128(void)
     return f;
 }
 
+/* ------------------------------------------------------- scale formats */
+/*
+ * UE8M0 scale (an 8-bit exponent, no mantissa: a power of two).  The review
+ * of [DSA] asks for a use_ue8m0 option of the 1x128 quantizer; the pages give
+ * no rounding rule.  Reading: the FP32 scale s of the FP8 rule is rounded up
+ * to the smallest power of two not below it (s itself when it is one), so no
+ * value quantizes above E4M3's largest (|y| / s_ue <= |y| / s <= 448, up to
+ * the rounding of s); +inf stays +inf.  The stored scale is that FP32 power
+ * of two; its UE8M0 byte is the binary32 exponent field (bits 30..23).
+ */
+static float ue8m0_ceil(float s)
+{
+    if (!(s > 0.0f) || isinf(s))
+        return s;
+    int e;
+    const float f = frexpf(s, &e); /* s = f * 2^e, f in [0.5, 1) */
+    return f == 0.5f ? s : ldexpf(1.0f, e);
+}
+
+/*
+ * Interleaved block-scale layout read by block-scaled tcgen05 MMAs (the
+ * layout DeepGEMM issue #320's discussion of tcgen05 data paths refers to;
+ * the pages print no formula).  Reading: a scale matrix of R rows (a
+ * multiple of 128) and C columns (a multiple of 4) is cut into tiles of 128
+ * rows x 4 columns, stored tile-row major (tile (R/128 index, C/4 index) at
+ * byte 512 * (tr * C/4 + tc)); inside a tile, element (r, c) sits at byte
+ * 16 * (r % 32) + 4 * (r / 32) + c, i.e. 32 lines of 16 bytes, line i holding
+ * rows i, i + 32, i + 64, i + 96, four scales each.
+ */
+static int64_t sf_swizzled(int64_t r, int64_t c, int64_t C)
+{
+    return ((r / 128) * (C / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4;
+}
+
+int64_t hqo_sf_swizzled_offset(int64_t r, int64_t c, int64_t C)
+{
+    return sf_swizzled(r, c, C);
+}
+
 /* ---------------------------------------------------------------- FP8 1xN */
 /*
  * One group of n values -> n E4M3 codes and one FP32 scale, as [QMOE] states:
@@ -189,13 +233,16 @@ static float c128(void)
  * rounded IEEE division.  `pre`, when given, receives y_i / s (the value that
  * is rounded to E4M3); `amax_out`, when given, receives amax.
  */
-static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, float *amax_out, float *pre)
+static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, float *amax_out, float *pre,
+                            int ue8m0)
 {
     float amax = 0.0f;
     for (int i = 0; i < n; ++i)
         amax = fmaxf(amax, fabsf(y[i]));
     const float inv448 = 1.0f / 448.0f; /* binary32 constant, 0x3B124925 */
     float s = fmaxf(amax, 1e-10f) * inv448;
+    if (ue8m0)
+        s = ue8m0_ceil(s);  /* y / s is then exact (a power of two), unless it underflows */
     for (int i = 0; i < n; ++i) {
         float t = y[i] / s;
         if (pre)
@@ -216,7 +263,8 @@ static void quant_group_fp8(const float *y, int n, uint8_t *q, float *scale, flo
  * Output codes: out[(t * G + g) * 128 + j].  Scales: scale_layout 0 (row
  * major) puts group (t, g) at scales[t * G + g]; layout 1 (transposed, as the
  * indexer stores them) at scales[g * scale_ld + t].  amax_opt, when given,
- * receives each group's amax in the scales' layout.
+ * receives each group's amax in the scales' layout.  scale_layout may add
+ * 256: UE8M0 scales (ue8m0_ceil).
  * Returns 0, or -1 for arguments this reference does not accept.
  */
 int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
@@ -225,6 +273,8 @@ int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
                        uint8_t *out, float *scales, int scale_layout, int64_t scale_ld,
                        float *amax_opt, float *pre)
 {
+    const int ue8m0 = (scale_layout & 256) != 0;
+    scale_layout &= ~256;
     if (a_width < 0 || b_width < 0 || a_width + b_width != 128 || (b_width > 0 && !b))
         return -1;
     if (hadamard_n != 0 && hadamard_n != 128)
@@ -244,7 +294,7 @@ int hqo_cat_rotate_fp8(const uint16_t *a, int64_t a_row_stride, int a_width,
             }
             int64_t grp = t * G + g;
             float s, am;
-            quant_group_fp8(v, 128, out + grp * 128, &s, &am, pre ? pre + grp * 128 : 0);
+            quant_group_fp8(v, 128, out + grp * 128, &s, &am, pre ? pre + grp * 128 : 0, ue8m0);
             const int64_t si = scale_layout == 0 ? grp : (int64_t)g * scale_ld + t;
             scales[si] = s;
             if (amax_opt)
@@ -330,11 +380,13 @@ static float swiglu(float g, float u)
  *           K_out..2*K_out-1 ("2x2048": the reading is two halves, not an
  *           interleave); the quantized value is SiLU(gate) * up.
  * out: [M, K_out] codes; scales (and amax_opt, when given, each group's
- * amax): [M, K_out/128] row major.
+ * amax): [M, K_out/128] row major.  mode may add 256: UE8M0 scales.
  */
 int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
                         uint8_t *out, float *scales, float *amax_opt, float *pre)
 {
+    const int ue8m0 = (mode & 256) != 0;
+    mode &= ~256;
     if (K_out % 128 != 0 || mode < 0 || mode > 2)
         return -1;
     const int64_t groups = K_out / 128;
@@ -354,7 +406,7 @@ int hqo_swiglu_fp8_k128(int mode, const void *in, int64_t M, int64_t K_out,
             }
             int64_t grp = m * groups + g;
             quant_group_fp8(y, 128, out + grp * 128, &scales[grp], amax_opt ? &amax_opt[grp] : 0,
-                            pre ? pre + grp * 128 : 0);
+                            pre ? pre + grp * 128 : 0, ue8m0);
         }
     return 0;
 }
@@ -532,6 +584,11 @@ static void rht16(const float *x, uint16_t sign_mask, float *v)
  *   offset + e of the stream of seed (rowwise) or seed + 1 (columnwise), e
  *   the element's index in its output (r*K + c rowwise; the index inside
  *   col_codes' element order columnwise).  Block scales stay nearest-even.
+ * flags bit 7 (128, scale layout for block-scaled MMAs): row_sf and each
+ *   section's col_sf block are stored in the interleaved 128 x 4 tiles of
+ *   sf_swizzled (rows M and K, columns K/16 and M_s/16: all multiples of the
+ *   tile, so the layout is a permutation of the plain one, section by
+ *   section).
  * row_pre / col_pre, when given, receive the value rounded to E2M1 per
  * element, in the output's layout.
  */
@@ -588,7 +645,7 @@ int hqo_group_rht_quant_sr(const uint16_t *x, int64_t M, int64_t K,
                         for (int i = 0; i < 16; ++i)
                             rnd[i] = sr_byte(seed, offset + (uint64_t)(r * K + kb * 16 + i));
                     nvfp4_block_r(rotate ? v : blk, S_enc, row_codes + r * (K / 2) + kb * 8,
-                                  row_sf + r * (K / 16) + kb,
+                                  row_sf + ((flags & 128) ? sf_swizzled(r, kb, K / 16) : r * (K / 16) + kb),
                                   row_pre ? row_pre + r * K + kb * 16 : 0, (flags & 32) ? rnd : 0);
                 }
         }
@@ -619,7 +676,8 @@ int hqo_group_rht_quant_sr(const uint16_t *x, int64_t M, int64_t K,
                     if (flags & 64)  /* element of col_codes: stream of seed + 1 */
                         for (int i = 0; i < 16; ++i)
                             rnd[i] = sr_byte(seed + 1, offset + (uint64_t)(K * r0 + c * Ms + mb * 16 + i));
-                    nvfp4_block_r(v, S_enc, cc + c * (Ms / 2) + mb * 8, cs + c * (Ms / 16) + mb,
+                    nvfp4_block_r(v, S_enc, cc + c * (Ms / 2) + mb * 8,
+                                  cs + ((flags & 128) ? sf_swizzled(c, mb, Ms / 16) : c * (Ms / 16) + mb),
                                   col_pre ? col_pre + K * r0 + c * Ms + mb * 16 : 0, (flags & 64) ? rnd : 0);
                 }
         }
@@ -656,7 +714,8 @@ int hqo_group_rht_quant(const uint16_t *x, int64_t M, int64_t K,
  *   (nvfp4_block), the vector's decode scale 1/S_enc stored like the FP8
  *   scales (row major [M, G] or transposed [G, scale_ld]).
  * codes: [M, G*64] bytes (vector (t, g) at (t*G + g)*64, element 2k in the
- * low nibble); block_sf: [M, G*8] E4M3 codes; amax_opt: A per vector in the
+ * low nibble); block_sf: [M, G*8] E4M3 codes (scale_layout + 128: the
+ * interleaved tiles of sf_swizzled, M a multiple of 128); amax_opt: A per vector in the
  * scales' layout; pre: the value rounded to E2M1 per element, [M, G*128].
  * Returns 0, or -1 for arguments this reference does not accept.
  */
@@ -666,6 +725,10 @@ int hqo_cat_rotate_nvfp4(const uint16_t *a, int64_t a_row_stride, int a_width,
                          uint8_t *codes, uint8_t *block_sf, float *sdec, int scale_layout, int64_t scale_ld,
                          float *amax_opt, float *pre)
 {
+    const int swz = (scale_layout & 128) != 0;
+    scale_layout &= ~128;
+    if (swz && M % 128 != 0)
+        return -1;
     if (a_width < 0 || b_width < 0 || a_width + b_width != 128 || (b_width > 0 && !b))
         return -1;
     if (hadamard_n != 0 && hadamard_n != 128)
@@ -689,7 +752,8 @@ int hqo_cat_rotate_nvfp4(const uint16_t *a, int64_t a_row_stride, int a_width,
             const float S_enc = global_encode_scale(A);
             const int64_t vec = t * G + g;
             for (int blk = 0; blk < 8; ++blk)
-                nvfp4_block(v + 16 * blk, S_enc, codes + vec * 64 + 8 * blk, block_sf + vec * 8 + blk,
+                nvfp4_block(v + 16 * blk, S_enc, codes + vec * 64 + 8 * blk,
+                            block_sf + (swz ? sf_swizzled(t, (int64_t)g * 8 + blk, (int64_t)G * 8) : vec * 8 + blk),
                             pre ? pre + vec * 128 + 16 * blk : 0);
             const int64_t si = scale_layout == 0 ? vec : (int64_t)g * scale_ld + t;
             sdec[si] = 1.0f / S_enc;

@@ -397,3 +397,36 @@ def test_status_codes(hq):
     for n, name in names.items():
         const = "HQ_OK" if name == "OK" else "HQ_ERR_" + name
         assert getattr(hq, const) == n
+
+
+# ------------------------------------------------------------- scale formats
+def test_ue8m0_bits_expression():
+    (expr,) = re.findall(r"`([^`]*)`", " ".join(r[1] for r in table_rows(section("6.4 Scale formats"))[:1]))
+    rng = np.random.default_rng(9)
+    M, G = 4, 2
+    pe = S.normal_bf16(401, (M, G, 64))
+    nope = S.with_outliers_bf16(S.normal_bf16(402, (M, G, 64)), 403, p=0.05, factor=300.0)
+    _, s_pl, _ = oracle.cat_rotate_fp8(pe, nope, M, G, 128)
+    _, s_ue, _ = oracle.cat_rotate_fp8(pe, nope, M, G, 128, scale_layout=oracle.UE8M0)
+    vals = list(s_pl.reshape(-1)) + [F(1.0), F(0.75), F(3e38), F(np.inf)] + list(
+        (rng.random(200) * np.exp2(rng.integers(-60, 60, 200))).astype(np.float32))
+    for v in vals:
+        got = ev(expr, bits=lambda x: bits(x), s=F(v)) & 0xFFFFFFFF
+        m, e = np.frexp(np.float64(v))
+        want = float(v) if (m == 0.5 or not np.isfinite(v)) else float(np.float32(np.ldexp(1.0, int(e))))
+        assert float(f32_of(got)) == want, (float(v), hex(got))
+    for a, b in zip(s_pl.reshape(-1), s_ue.reshape(-1)):
+        assert bits(b) == ev(expr, bits=lambda x: bits(x), s=F(a)) & 0xFFFFFFFF
+
+
+def test_interleaved_scale_offsets():
+    rows = table_rows(section("6.4 Scale formats"))
+    (expr,) = re.findall(r"`([^`]*)`", [r for r in rows if r[0] == "interleaved scales"][0][2])
+    for R, C in ((128, 8), (256, 16), (384, 28)):
+        seen = set()
+        for r in range(R):
+            for c in range(C):
+                o = ev(expr, r=r, c=c, C=C)
+                assert o == oracle.sf_swizzled_offset(r, c, C)
+                seen.add(o)
+        assert seen == set(range(R * C))
