@@ -60,8 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="grouped_moe",
-                    choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr", "dense_nvfp4",
-                             "dsa_indexer", "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
+                    choices=("grouped_moe", "grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr",
+                             "grouped_moe_sf_interleaved", "dense_nvfp4", "dsa_indexer", "dsa_indexer_ue8m0",
+                             "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"))
     ap.add_argument("--no-extras", action="store_true", help="time only the headline workload")
     ap.add_argument("--schedule", choices=("fused", "two_pass"), default="fused")
     ap.add_argument("--no-e2e", action="store_true")
@@ -384,6 +385,29 @@ class GroupedNVFP4(Workload):
                 f"on {cores} threads")
 
 
+class GroupedInterleavedSF(GroupedNVFP4):
+    """The grouped cast with its block scales in the interleaved 128 x 4 tiles
+    block-scaled tcgen05 MMAs read (HQ_SF_SWIZZLED)."""
+    name = "grouped_moe_sf_interleaved"
+    host_pipeline = False
+
+    def config(self):
+        c = super().config()
+        c["workload"] += ", block scales in interleaved 128x4 tiles"
+        return c
+
+    def flags(self):
+        return super().flags() | self.hq.HQ_SF_SWIZZLED
+
+    def oracle_sample(self, host, rows=512):
+        import oracle
+        x = host["x"][:rows]
+        flags = oracle.ROWWISE | oracle.COLWISE | oracle.SF_SWIZZLED
+        return (lambda: oracle.group_rht_quant(x, [rows], self.mask, flags),
+                rows * self.K * 2 + 2 * (rows * self.K // 2 + rows * self.K // 16),
+                f"one {rows}-row section of the BF16 [{self.M},{self.K}] input, interleaved block scales")
+
+
 class GroupedAmaxGiven(GroupedNVFP4):
     """The same workload with the section amax values supplied by the caller
     (HQ_AMAX_GIVEN): one pass over x.  The amax values come from one ordinary
@@ -562,6 +586,28 @@ class DSAIndexerNVFP4(DSAIndexer):
                 f"tokens 0..{tokens - 1} of the [{self.T},{self.H}] indexer input")
 
 
+class DSAIndexerUE8M0(DSAIndexer):
+    """The indexer prep with UE8M0 (power-of-two) FP8 scales."""
+    name = "dsa_indexer_ue8m0"
+
+    def config(self):
+        c = super().config()
+        c["workload"] += ", UE8M0 scales"
+        return c
+
+    def call(self, inputs, out):
+        hq = self.hq
+        hq.hq_cat_rotate_fp8(inputs["pe"], self.H * 64, 64, inputs["nope"], self.H * 64, 64, self.T, self.H,
+                             128, out["codes"], out["scales"], hq.HQ_SCALE_TRANSPOSED | hq.HQ_FP8_UE8M0, self.T)
+
+    def oracle_sample(self, host, tokens=256):
+        import oracle
+        pe, nope = host["pe"][:tokens], host["nope"][:tokens]
+        return (lambda: oracle.cat_rotate_fp8(pe, nope, tokens, self.H, 128,
+                                              scale_layout=oracle.TRANSPOSED | oracle.UE8M0, scale_ld=tokens),
+                tokens * self.H * (128 * 3 + 4), f"tokens 0..{tokens - 1} of the [{self.T},{self.H}] indexer input")
+
+
 class FP8Single(DSAIndexer):
     name = "fp8_single"
 
@@ -641,6 +687,8 @@ class QMoE(Workload):
 def make_workload(name: str, rank: int, schedule: str = "fused") -> Workload:
     return {"grouped_moe": lambda: GroupedNVFP4(rank, schedule=schedule),
             "grouped_moe_amax_given": lambda: GroupedAmaxGiven(rank),
+            "grouped_moe_sf_interleaved": lambda: GroupedInterleavedSF(rank, schedule=schedule),
+            "dsa_indexer_ue8m0": lambda: DSAIndexerUE8M0(rank),
             "grouped_moe_row_rht": lambda: GroupedRowRHT(rank, schedule=schedule),
             "grouped_moe_sr": lambda: GroupedSR(rank, schedule=schedule),
             "dense_nvfp4": lambda: DenseNVFP4(rank, schedule=schedule),
@@ -921,8 +969,9 @@ def run_ours(args, ranks: Ranks) -> None:
         del main, host_main
         torch.cuda.empty_cache()
         extras = {}
-        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr", "dense_nvfp4", "dsa_indexer",
-                     "dsa_indexer_nvfp4", "qmoe_bf16", "qmoe_swiglu", "fp8_single"):
+        for name in ("grouped_moe_amax_given", "grouped_moe_row_rht", "grouped_moe_sr", "grouped_moe_sf_interleaved",
+                     "dense_nvfp4", "dsa_indexer", "dsa_indexer_ue8m0", "dsa_indexer_nvfp4", "qmoe_bf16",
+                     "qmoe_swiglu", "fp8_single"):
             if name == args.workload:
                 continue
             r = measure(torch, hq, name, args, ranks, flush)

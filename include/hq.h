@@ -62,6 +62,9 @@ typedef enum hq_status {
 #define HQ_COL_SR 64u      /* hq_group_rht_quant_sr: columnwise codes round stochastically */
 #define HQ_AMAX_GIVEN 16u  /* amax_row / amax_col are inputs: the caller's section
                               amax values; one pass, no amax computation */
+#define HQ_SF_SWIZZLED 128u /* row_sf and each section's col_sf block in the
+                              interleaved 128 x 4 tiles that block-scaled
+                              tcgen05 MMAs read (see below) */
 #define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
                               instead of one launch in which each section's
                               cast follows its amax while the rows are still
@@ -71,7 +74,30 @@ typedef enum hq_status {
 #define HQ_SCALE_ROWMAJOR 0   /* scale of group (t, g) at scales[t * G + g] */
 #define HQ_SCALE_TRANSPOSED 1 /* scale of group (t, g) at scales[g * scale_ld + t] */
 
-/* hq_swiglu_fp8_k128 modes */
+/*
+ * Scale formats for GEMMs that consume the outputs directly (the TensorRT-LLM
+ * PR #15158 review asks for a use_ue8m0 option of the 1x128 quantizer;
+ * DeepGEMM issue #320 discusses the tcgen05 data-path layouts of scales).
+ *
+ * HQ_FP8_UE8M0, added to scale_layout of hq_cat_rotate_fp8 or to mode of
+ * hq_swiglu_fp8_k128: each group's FP32 scale s is rounded up to the smallest
+ * power of two not below it, and the codes are E4M3(y / that power of two).
+ * The stored scale is that FP32 power of two; its UE8M0 byte is the binary32
+ * exponent field (bits 30..23).
+ *
+ * HQ_SF_SWIZZLED (hq_group_rht_quant* flags; added to scale_layout of
+ * hq_cat_rotate_nvfp4): E4M3 block scales in tiles of 128 rows x 4 columns
+ * of the [rows, cols] scale matrix, 512 bytes each, stored tile-row major;
+ * element (r, c) at byte
+ *   ((r / 128) * (cols / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+ * The grouped cast's row_sf is [M, K/16]; each section's col_sf block is
+ * [K, M_s/16] at its usual byte K * r0 / 16 (every dimension a multiple of the
+ * tile: a permutation of the plain layout, same size).  The FP4 DSA call's
+ * block_sf is [M, G * 8] and needs M % 128 == 0 (HQ_ERR_ALIGN otherwise).
+ */
+#define HQ_FP8_UE8M0 256
+
+/* hq_swiglu_fp8_k128 modes (+ HQ_FP8_UE8M0) */
 #define HQ_ACT_NONE_BF16 0  /* in: BF16 [M, K_out] */
 #define HQ_ACT_NONE_F32 1   /* in: FP32 [M, K_out] */
 #define HQ_ACT_SWIGLU_F32 2 /* in: FP32 [M, 2*K_out], gate = cols [0, K_out),
@@ -131,7 +157,8 @@ hq_status hq_get_error(void *ws, size_t ws_bytes, uint32_t *err_out, void *strea
  *  flags      HQ_ROWWISE | HQ_COLWISE (at least one), optionally HQ_ROW_RHT
  *             (only with HQ_ROWWISE; the grouped-quant pages speak of the RHT
  *             on both outputs, their fused kernel rotates only the columns),
- *             HQ_AMAX_GIVEN and HQ_TWO_PASS (ignored with HQ_AMAX_GIVEN).
+ *             HQ_AMAX_GIVEN, HQ_TWO_PASS (ignored with HQ_AMAX_GIVEN) and
+ *             HQ_SF_SWIZZLED.
  *
  * For section s (rows [r0, r0 + M_s)) and each requested direction:
  *   A_s = max |v| over the section's values (v = x rowwise, the RHT16 output
@@ -288,7 +315,8 @@ hq_status hq_group_rht_quant_noalloc(const void *x, int64_t M, int64_t K,
  *  scales     float: group scale s = max(amax, 1e-10) * float32(1/448),
  *             codes = E4M3(y / s) (IEEE division, saturating RNE).
  *             scale_layout HQ_SCALE_ROWMAJOR: [M, G] (scale_ld ignored);
- *             HQ_SCALE_TRANSPOSED: [G, scale_ld], scale_ld >= M.
+ *             HQ_SCALE_TRANSPOSED: [G, scale_ld], scale_ld >= M; either may
+ *             add HQ_FP8_UE8M0.
  *  amax_opt   float, NULL or each group's amax = max |y| (y the rotated
  *             128-vector), in the scales' layout; 4-byte aligned.
  *  ws, ws_bytes  unused: hq_cat_rotate_fp8_workspace_size() is 0 (may be
@@ -328,7 +356,8 @@ size_t hq_cat_rotate_fp8_workspace_size(void);
  *  amax_opt   float, NULL or A per vector, in the same layout.
  *  ws, ws_bytes  unused: hq_cat_rotate_nvfp4_workspace_size() is 0.
  * Errors: HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_UNSUPPORTED,
- *         HQ_ERR_CUDA.  Inputs must be finite.
+ *         HQ_ERR_CUDA.  Inputs must be finite.  scale_layout may add
+ *         HQ_SF_SWIZZLED (block_sf in the interleaved tiles, M % 128 == 0).
  */
 hq_status hq_cat_rotate_nvfp4(const void *a, int64_t a_row_stride, int a_width,
                               const void *b, int64_t b_row_stride, int b_width,
@@ -345,7 +374,8 @@ size_t hq_cat_rotate_nvfp4_workspace_size(void);
  * split into consecutive groups of 128; each group gets the FP8 rule above.
  *  mode     HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32 or HQ_ACT_SWIGLU_F32 (the value
  *           quantized is SiLU(gate) * up computed in FP32, SiLU(g) =
- *           g / (1 + exp(-g)), with no narrower rounding in between).
+ *           g / (1 + exp(-g)), with no narrower rounding in between); any
+ *           mode may add HQ_FP8_UE8M0.
  *  in       see the modes; row stride K_out (or 2*K_out for SwiGLU).
  *  out_fp8  uint8 [M, K_out];  scales float [M, K_out/128] row major.
  *  amax_opt float [M, K_out/128] or NULL: each group's amax = max |y|.

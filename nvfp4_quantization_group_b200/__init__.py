@@ -24,6 +24,7 @@ HQ_OK, HQ_ERR_NULL, HQ_ERR_SHAPE, HQ_ERR_ALIGN, HQ_ERR_WORKSPACE, HQ_ERR_UNSUPPO
     HQ_ERR_TIMEOUT = range(8)
 HQ_ROWWISE, HQ_COLWISE, HQ_ROW_RHT, HQ_TWO_PASS, HQ_AMAX_GIVEN, HQ_ROW_SR, HQ_COL_SR = 1, 2, 4, 8, 16, 32, 64
 HQ_SCALE_ROWMAJOR, HQ_SCALE_TRANSPOSED = 0, 1
+HQ_SF_SWIZZLED, HQ_FP8_UE8M0 = 128, 256  # scale formats (see include/hq.h)
 HQ_ACT_NONE_BF16, HQ_ACT_NONE_F32, HQ_ACT_SWIGLU_F32 = 0, 1, 2
 HQ_FMT_E4M3, HQ_FMT_E2M1 = 0, 1
 HQ_MAX_SECTIONS = 256
@@ -345,7 +346,7 @@ def cat_rotate_fp8(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 12
     M, G, aw = a.shape
     bw = 0 if b is None else b.shape[-1]
     codes = torch.empty((M, G * 128), dtype=torch.uint8, device=a.device)
-    if scale_layout == HQ_SCALE_ROWMAJOR:
+    if (scale_layout & ~HQ_FP8_UE8M0) == HQ_SCALE_ROWMAJOR:
         scales = torch.empty((M, G), dtype=torch.float32, device=a.device)
         ld = G
     else:
@@ -367,7 +368,7 @@ def cat_rotate_nvfp4(a: torch.Tensor, b: torch.Tensor | None, hadamard_n: int = 
     dev = a.device
     out = {"codes": torch.empty((M, G * 64), dtype=torch.uint8, device=dev),
            "block_sf": torch.empty((M, G * 8), dtype=torch.uint8, device=dev)}
-    if scale_layout == HQ_SCALE_ROWMAJOR:
+    if (scale_layout & ~HQ_SF_SWIZZLED) == HQ_SCALE_ROWMAJOR:
         out["sdec"] = torch.empty((M, G), dtype=torch.float32, device=dev)
         ld = G
     else:

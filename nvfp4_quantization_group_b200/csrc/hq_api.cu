@@ -181,7 +181,7 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
                                  float* amax_row, float* amax_col, float* sdec_row, float* sdec_col, void* ws,
                                  size_t ws_bytes, void* stream) {
     // ---- argument checks (nothing is launched on failure)
-    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR))
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR | HQ_SF_SWIZZLED))
         return HQ_ERR_UNSUPPORTED;
     if ((flags & HQ_ROW_SR) && !(flags & HQ_ROWWISE)) return HQ_ERR_UNSUPPORTED;
     if ((flags & HQ_COL_SR) && !(flags & HQ_COLWISE)) return HQ_ERR_UNSUPPORTED;
@@ -224,7 +224,7 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
     p.ws = static_cast<uint32_t*>(ws);
     p.S = S;
     p.sign_mask = sign_mask;
-    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_ROW_SR | HQ_COL_SR);
+    p.flags = flags & (HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_ROW_SR | HQ_COL_SR | HQ_SF_SWIZZLED);
     p.sr_seed = sr_seed;
     p.sr_offset = sr_offset;
     p.col_tiles = (int)(K / NV_TILE);
@@ -349,7 +349,7 @@ hq_status hq_group_rht_quant_host(const void* x, int64_t M, int64_t K, const int
                                   void* h2d_stream, void* d2h_stream) {
     // ---- checks of what the per-group calls cannot see (they check the rest
     // again on the staging pointers)
-    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR))
+    if (flags & ~(HQ_ROWWISE | HQ_COLWISE | HQ_ROW_RHT | HQ_AMAX_GIVEN | HQ_TWO_PASS | HQ_ROW_SR | HQ_COL_SR | HQ_SF_SWIZZLED))
         return HQ_ERR_UNSUPPORTED;
     const bool do_row = flags & HQ_ROWWISE, do_col = flags & HQ_COLWISE;
     if (!do_row && !do_col) return HQ_ERR_UNSUPPORTED;
@@ -472,6 +472,10 @@ static hq_status cat_rotate(const void* a, int64_t a_row_stride, int a_width, co
                             int b_width, int64_t M, int G, int hadamard_n, uint8_t* out, uint8_t* sf, float* scales,
                             int scale_layout, int64_t scale_ld, float* amax_opt, void* stream, bool fp4) {
     if (hadamard_n != 0 && hadamard_n != 128) return HQ_ERR_UNSUPPORTED;
+    // the format bit of this call: UE8M0 FP8 scales, or interleaved FP4 block scales
+    const int fmt_bit = fp4 ? (int)HQ_SF_SWIZZLED : HQ_FP8_UE8M0;
+    const bool fmt = (scale_layout & fmt_bit) != 0;
+    scale_layout &= ~fmt_bit;
     if (scale_layout != HQ_SCALE_ROWMAJOR && scale_layout != HQ_SCALE_TRANSPOSED) return HQ_ERR_UNSUPPORTED;
     if (M < 0 || G <= 0 || a_width < 0 || b_width < 0 || a_width + b_width != 128) return HQ_ERR_SHAPE;
     if (M == 0) return HQ_OK;
@@ -480,6 +484,7 @@ static hq_status cat_rotate(const void* a, int64_t a_row_stride, int a_width, co
     if (a_row_stride < (int64_t)G * a_width || (b_width > 0 && b_row_stride < (int64_t)G * b_width))
         return HQ_ERR_SHAPE;
     if (scale_layout == HQ_SCALE_TRANSPOSED && scale_ld < M) return HQ_ERR_SHAPE;
+    if (fp4 && fmt && M % 128 != 0) return HQ_ERR_ALIGN;  // whole 128-row tiles of block scales
     if (!aligned16(a) || (b_width > 0 && !aligned16(b)) || !aligned16(out) || !aligned4(scales) ||
         !aligned4(amax_opt))
         return HQ_ERR_ALIGN;
@@ -503,6 +508,8 @@ static hq_status cat_rotate(const void* a, int64_t a_row_stride, int a_width, co
     p.amax = amax_opt;
     p.scale_layout = scale_layout;
     p.scale_ld = scale_ld;
+    p.ue8m0 = !fp4 && fmt;
+    p.sf_swizzle = fp4 && fmt;
     p.wide = a_width % 16 == 0 && b_width % 16 == 0 && a_row_stride % 16 == 0 && b_row_stride % 16 == 0 &&
              (reinterpret_cast<uintptr_t>(a) & 31u) == 0 && (b_width == 0 || (reinterpret_cast<uintptr_t>(b) & 31u) == 0);
     p.ntiles = cat_rotate_tiles(p);
@@ -542,6 +549,8 @@ hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out,
                              float* scales, float* amax_opt, void* ws, size_t ws_bytes, void* stream) {
     (void)ws;
     (void)ws_bytes;
+    const bool ue8m0 = (mode & HQ_FP8_UE8M0) != 0;
+    mode &= ~HQ_FP8_UE8M0;
     if (mode != HQ_ACT_NONE_BF16 && mode != HQ_ACT_NONE_F32 && mode != HQ_ACT_SWIGLU_F32) return HQ_ERR_UNSUPPORTED;
     if (M < 0 || K_out <= 0) return HQ_ERR_SHAPE;
     if (K_out % 128) return HQ_ERR_ALIGN;
@@ -558,6 +567,7 @@ hq_status hq_swiglu_fp8_k128(int mode, const void* in, int64_t M, int64_t K_out,
     p.gpr_magic = 0xFFFFFFFFu / (uint32_t)(K_out / 128);
     p.out = out_fp8;
     p.scales = scales;
+    p.ue8m0 = ue8m0 ? 1 : 0;
     p.amax = amax_opt;
     constexpr int warps_per_block = K128_THREADS / 32;
     const int64_t pairs = (p.ngroups + 1) / 2;

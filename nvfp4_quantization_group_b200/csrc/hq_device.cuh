@@ -106,6 +106,21 @@ __device__ __forceinline__ float fp8_group_scale(float amax) {
     return __fmul_rn(fmaxf(amax, floor_), inv448);
 }
 
+// The smallest power of two not below s > 0 (UE8M0 scale; +inf stays +inf):
+// adding 2^23 - 1 to the bits carries into the exponent unless the mantissa
+// is zero, then the mantissa is cleared.
+__device__ __forceinline__ float ue8m0_up(float s) {
+    return __uint_as_float((__float_as_uint(s) + 0x7FFFFFu) & 0xFF800000u);
+}
+
+// Byte offset of element (r, c) of a block-scale matrix with `cols` columns
+// in the interleaved tiles of 128 rows x 4 columns (512 bytes, tile-row major;
+// inside a tile line r % 32 of 16 bytes holds rows r % 32 + 32 i, 4 scales
+// each).
+__device__ __forceinline__ uint64_t sf_swizzled(uint64_t r, uint64_t c, uint64_t cols) {
+    return ((r >> 7) * (cols >> 2) + (c >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (c & 3u);
+}
+
 // ----------------------------------------------- correctly rounded y / b
 // The quantizers divide many numerators by one divisor b.  Instead of an
 // IEEE division per element they take r = RN(1/b) once and refine

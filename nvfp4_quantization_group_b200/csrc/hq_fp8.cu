@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
                 *reinterpret_cast<uint2*>(p.out + v * 64 + 8 * j) =
                     make_uint2(e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]),
                                e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]));
-                p.sf[v * 8 + j] = (uint8_t)sf;
+                p.sf[p.sf_swizzle ? sf_swizzled((uint64_t)cv.t, (uint64_t)cv.g * 8u + (uint64_t)j, (uint64_t)p.G * 8u)
+                                  : (uint64_t)v * 8u + (uint64_t)j] = (uint8_t)sf;
                 if (j == 0) {
                     const int64_t si = p.scale_layout == 0 ? v : (int64_t)cv.g * p.scale_ld + cv.t;
                     p.scales[si] = __fdiv_rn(1.0f, S);
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
             __syncwarp();  // the exchange buffer is reused by the next tile
             continue;
         }
-        const float sc = fp8_group_scale(amax);
+        const float sc = p.ue8m0 ? ue8m0_up(fp8_group_scale(amax)) : fp8_group_scale(amax);
         // ---- codes of elements 16s + 2j, 16s + 2j + 1
         uint32_t q[8];
         if (!isinf(sc)) {
@@ -380,7 +381,7 @@ __device__ __forceinline__ void k128_finish(const K128Params& p, uint32_t g, boo
     }
 #pragma unroll
     for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const float s = fp8_group_scale(m);
+    const float s = p.ue8m0 ? ue8m0_up(fp8_group_scale(m)) : fp8_group_scale(m);
     if (valid) {
         const uint2 c = quant8(ny, s);
         uint8_t* out = p.out + (uint64_t)g * 128;

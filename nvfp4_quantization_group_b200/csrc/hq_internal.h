@@ -31,6 +31,8 @@ struct CatRotateParams {
     float* amax;  // NULL or per-group amax, in the scales' layout
     int scale_layout;
     int64_t scale_ld;
+    int ue8m0;       // FP8: scales rounded up to powers of two
+    int sf_swizzle;  // FP4: block scales in the interleaved 128 x 4 tiles
 };
 
 struct K128Params {
@@ -41,6 +43,7 @@ struct K128Params {
     uint8_t* out;
     float* scales;
     float* amax;  // NULL or per-group amax [M, K_out / 128]
+    int ue8m0;    // scales rounded up to powers of two
 };
 
 constexpr int K128_THREADS = 256;   // 8 warps, two K128 groups per warp step

@@ -586,6 +586,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         uint32_t coff;     // columnwise: pair 4 vw + jw, row 16 rb
         int cpair;         //   first of its two columns, inside the tile
         uint64_t rs_off0;  // row rr's block-scale offset (+ 4 K16 for rr + 4; codes at 8x)
+        uint32_t rs_swz;   // the same inside the tile's 1 KB of interleaved row scales (+ 64 for rr + 4)
+        uint32_t cs_swz;   // column cpair's scale of row block rb inside the tile's 1 KB of
+                           //   interleaved column scales (+ 16 for cpair + 1)
     };
     // This lane's two rows (rr, rr + 4) of part pt in element order: lanes with
     // `swap` loaded the odd chunk first.
@@ -610,6 +613,11 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         q.coff = chunk_off(vw >> 3, rb, 0, vw & 7) + 4u * (uint32_t)jw;  // chunk vw & 7 of half vw >> 3
         q.cpair = 8 * vw + 2 * jw;
         q.rs_off0 = (uint64_t)rr * K16 + b;
+        // interleaved tiles: a 128-row x 128-column tile of x owns two whole
+        // 128 x 4 scale tiles per direction (1 KB); rr + 4 and cpair + 1 stay
+        // in the same 32-row line group
+        q.rs_swz = (uint32_t)((b >> 2) * 512 + (rr & 31) * 16 + (rr >> 5) * 4 + (b & 3));
+        q.cs_swz = (uint32_t)((rb >> 2) * 512 + (q.cpair & 31) * 16 + (q.cpair >> 5) * 4 + (rb & 3));
         return q;
     };
     Part parts[16 / NCW];  // the same for every tile
@@ -701,7 +709,11 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         } else if (!(h.flags & H_GAVE_UP)) {
             // ===================================================== cast tile
             uint8_t* const rc_base = p.row_codes + (uint64_t)h.row0 * K2 + (uint32_t)h.col0 / 2u;
-            uint8_t* const rs_base = p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
+            const bool swz = p.flags & HQ_SF_SWIZZLED;
+            // row scales: the plain [M, K/16] rows, or the tile's 1 KB of interleaved tiles
+            uint8_t* const rs_base = swz ? p.row_sf + (((uint64_t)h.row0 >> 7) * (K16 >> 2) + ((uint32_t)h.col0 >> 6)) * 512u
+                                         : p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
+            const uint64_t rs_4 = swz ? 64u : 4u * K16;  // row rr + 4
 #pragma unroll
             for (int pi = 0; pi < 16 / NCW; ++pi) {
             const Part& pt = parts[pi];
@@ -741,8 +753,9 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 }
                 *reinterpret_cast<uint2*>(rc_base + 8u * pt.rs_off0) = ca;
                 *reinterpret_cast<uint2*>(rc_base + 8u * (pt.rs_off0 + 4u * K16)) = cbw;
-                rs_base[pt.rs_off0] = (uint8_t)sf0;
-                rs_base[pt.rs_off0 + 4u * K16] = (uint8_t)sf1;
+                const uint64_t so = swz ? pt.rs_swz : pt.rs_off0;
+                rs_base[so] = (uint8_t)sf0;
+                rs_base[so + rs_4] = (uint8_t)sf1;
             } else if (do_row) {
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
@@ -776,7 +789,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                     }
                     *reinterpret_cast<uint2*>(rc_base + 8u * rs_off) =
                         swap ? make_uint2(c1, c0) : make_uint2(c0, c1);
-                    rs_base[rs_off] = (uint8_t)sf;
+                    rs_base[(swz ? pt.rs_swz : pt.rs_off0) + (kk ? rs_4 : 0u)] = (uint8_t)sf;
                 }
             }
             if (do_col) {
@@ -805,6 +818,11 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                 const uint64_t c = (uint32_t)(h.col0 + pt.cpair);
                 uint8_t* const cb = p.col_codes + (uint64_t)h.r0s * K2 + c * ms2 +
                                     ((uint32_t)h.row_in_sec0 / 2u + 8u * (uint32_t)rb);
+                // (interleaved: the section's [K, M_s/16] scales in 128 x 4 tiles; this
+                // tile of x owns 1 KB of them)
+                uint8_t* const sbz = p.col_sf + (uint64_t)h.r0s * K16 +
+                                     (((uint64_t)(uint32_t)h.col0 >> 7) * (ms16 >> 2) + ((uint32_t)h.row_in_sec0 >> 6)) * 512u +
+                                     pt.cs_swz;
                 uint8_t* const sb = p.col_sf + (uint64_t)h.r0s * K16 + c * ms16 +
                                     ((uint32_t)h.row_in_sec0 / 16u + (uint32_t)rb);
                 if (sr_col) {
@@ -823,8 +841,13 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
                         make_uint2(e2m1x8(q1[0], q1[1], q1[2], q1[3], q1[4], q1[5], q1[6], q1[7]),
                                    e2m1x8(q1[8], q1[9], q1[10], q1[11], q1[12], q1[13], q1[14], q1[15]));
                 }
-                sb[0] = (uint8_t)sf0;
-                sb[ms16] = (uint8_t)sf1;
+                if (swz) {
+                    sbz[0] = (uint8_t)sf0;
+                    sbz[16] = (uint8_t)sf1;
+                } else {
+                    sb[0] = (uint8_t)sf0;
+                    sb[ms16] = (uint8_t)sf1;
+                }
             }
             }  // parts
         }

@@ -85,7 +85,7 @@ def test_group_rht_quant_sr_argument_errors(L):
     assert _grp_sr(L, offset=8) == hq.HQ_ERR_ALIGN                        # offset % 16
     assert _grp_sr(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_SR) == hq.HQ_ERR_UNSUPPORTED
     assert _grp_sr(L, flags=hq.HQ_ROWWISE | hq.HQ_COL_SR) == hq.HQ_ERR_UNSUPPORTED
-    assert _grp_sr(L, flags=3 | 128) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_sr(L, flags=3 | 512) == hq.HQ_ERR_UNSUPPORTED
     assert _grp(L, x=0) == hq.HQ_ERR_NULL
     assert _grp(L, ws=0) == hq.HQ_ERR_NULL
     assert _grp(L, ptrs=0) == hq.HQ_ERR_NULL
@@ -118,7 +118,7 @@ def test_group_rht_quant_host_sizes_and_argument_errors(L):
     assert hq.hq_group_rht_quant_host_device_bytes(256, 256, 0) == 0
     assert hq.hq_group_rht_quant_host_device_bytes(-1, 256, 1) == 0
     assert _grp_host(L, flags=0) == hq.HQ_ERR_UNSUPPORTED
-    assert _grp_host(L, flags=3 | 128) == hq.HQ_ERR_UNSUPPORTED
+    assert _grp_host(L, flags=3 | 512) == hq.HQ_ERR_UNSUPPORTED
     assert _grp_host(L, flags=hq.HQ_COLWISE | hq.HQ_ROW_SR) == hq.HQ_ERR_UNSUPPORTED
     assert _grp_host(L, flags=3 | hq.HQ_COL_SR, offset=8) == hq.HQ_ERR_ALIGN
     assert _grp_host(L, split_ptr=False) == hq.HQ_ERR_NULL
@@ -160,6 +160,8 @@ def test_cat_rotate_fp8_argument_errors(L):
     assert call(layout=1, ld=8) == hq.HQ_ERR_SHAPE                 # transposed ld < M
     assert call(out=FAKE + 1) == hq.HQ_ERR_ALIGN
     assert call(amax=FAKE + 2) == hq.HQ_ERR_ALIGN
+    assert call(layout=hq.HQ_SF_SWIZZLED) == hq.HQ_ERR_UNSUPPORTED   # a format bit of the FP4 call
+    assert call(layout=1 | hq.HQ_FP8_UE8M0, ld=8) == hq.HQ_ERR_SHAPE  # UE8M0 keeps the layout's checks
     assert L.hq_cat_rotate_fp8_workspace_size() == 0
 
 
@@ -178,6 +180,8 @@ def test_cat_rotate_nvfp4_argument_errors(L):
     assert call(codes=FAKE + 8) == hq.HQ_ERR_ALIGN
     assert call(amax=FAKE + 2) == hq.HQ_ERR_ALIGN
     assert call(layout=1, ld=8) == hq.HQ_ERR_SHAPE
+    assert call(layout=hq.HQ_FP8_UE8M0) == hq.HQ_ERR_UNSUPPORTED     # a format bit of the FP8 calls
+    assert call(layout=hq.HQ_SF_SWIZZLED) == hq.HQ_ERR_ALIGN         # interleaved tiles need M % 128 == 0
     assert L.hq_cat_rotate_nvfp4_workspace_size() == 0
 
 
@@ -185,6 +189,9 @@ def test_swiglu_fp8_k128_argument_errors(L):
     def call(mode=0, inp=FAKE, M=4, K=256, out=FAKE, sc=FAKE, amax=None):
         return L.hq_swiglu_fp8_k128(mode, P(inp), M, K, P(out), P(sc), P(amax), None, 0, None)
     assert call(mode=3) == hq.HQ_ERR_UNSUPPORTED
+    assert call(mode=3 | hq.HQ_FP8_UE8M0) == hq.HQ_ERR_UNSUPPORTED
+    assert call(mode=hq.HQ_SF_SWIZZLED) == hq.HQ_ERR_UNSUPPORTED
+    assert call(mode=hq.HQ_FP8_UE8M0, K=200) == hq.HQ_ERR_ALIGN
     assert call(K=200) == hq.HQ_ERR_ALIGN
     assert call(M=-1) == hq.HQ_ERR_SHAPE
     assert call(M=0) == hq.HQ_OK

@@ -31,13 +31,14 @@ def _cat_case(hq, pe, nope, M, G, hadamard_n, layout, ld=None):
     want_c, want_s, _, want_a = oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, scale_layout=layout,
                                                       scale_ld=ld if layout else None, want_amax=True)
     got_s, got_a = scales.cpu().numpy(), amax.cpu().numpy()
-    if layout == oracle.TRANSPOSED:
+    if (layout & 1) == oracle.TRANSPOSED:
         got_s, want_s = got_s[:, :M], want_s[:, :M]
         got_a, want_a = got_a[:, :M], want_a[:, :M]
     assert_bits_equal(got_s, want_s, "scales")
     assert_bits_equal(got_a, want_a, "amax")
     assert_fp8_codes(codes.cpu().numpy(), want_c,
-                     lambda: oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, want_pre=True)[2])
+                     lambda: oracle.cat_rotate_fp8(pe, nope, M, G, hadamard_n, scale_layout=layout & oracle.UE8M0,
+                                                   want_pre=True)[2])
 
 
 def test_single_tensor_h128_fp8_512x128(hq):
@@ -81,6 +82,24 @@ def test_cat_zero_and_constant_vectors(hq):
     _cat_case(hq, pe, nope, M, G, 0, oracle.ROWMAJOR)
 
 
+@pytest.mark.parametrize("hadamard_n", [0, 128])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_cat_ue8m0_ragged_tokens_and_heads(hq, hadamard_n, layout):
+    """UE8M0 scales: powers of two, codes of y / 2^k."""
+    M, G = 37, 5
+    pe = S.normal_bf16(221, (M, G, 64))
+    nope = S.with_outliers_bf16(S.normal_bf16(222, (M, G, 64)), 223, p=0.01, factor=1e3)
+    _cat_case(hq, pe, nope, M, G, hadamard_n, layout | hq.HQ_FP8_UE8M0, ld=40 if layout else None)
+
+
+@pytest.mark.slow
+def test_dsa_indexer_ue8m0_full_4096x64(hq):
+    seed = S.SEEDS["dsa_indexer"]
+    pe = S.normal_bf16(seed, (4096, 64, 64))
+    nope = S.normal_bf16(seed + 100, (4096, 64, 64))
+    _cat_case(hq, pe, nope, 4096, 64, 128, oracle.TRANSPOSED | hq.HQ_FP8_UE8M0, ld=4096)
+
+
 @pytest.mark.slow
 def test_dsa_indexer_full_4096x64(hq):
     """Full DSA indexer prep: q_pe, q_nope [4096, 64, 64], transposed scales [64, 4096]."""
@@ -104,7 +123,7 @@ def _cat4_case(hq, pe, nope, M, G, hadamard_n, layout, ld=None):
                                    scale_ld=ld if layout else None, want_amax=True)
     for k in ("sdec", "amax"):
         g, w = got[k], want[k]
-        if layout == oracle.TRANSPOSED:
+        if (layout & 1) == oracle.TRANSPOSED:
             g, w = g[:, :M], w[:, :M]
         assert_bits_equal(g, w, k)
     assert_bits_equal(got["block_sf"], want["block_sf"], "block_sf")
@@ -142,6 +161,23 @@ def test_cat_nvfp4_magnitudes(hq):
     _cat4_case(hq, x[..., :64].copy(), x[..., 64:].copy(), M, G, 128, oracle.TRANSPOSED, ld=8)
 
 
+@pytest.mark.parametrize("layout", [0, 1])
+def test_cat_nvfp4_interleaved_block_scales(hq, layout):
+    """Block scales in the interleaved 128 x 4 tiles (M a multiple of 128)."""
+    M, G = 256, 3
+    pe = S.normal_bf16(271, (M, G, 64))
+    nope = S.with_outliers_bf16(S.normal_bf16(272, (M, G, 64)), 273, p=0.01)
+    _cat4_case(hq, pe, nope, M, G, 128, layout | hq.HQ_SF_SWIZZLED, ld=264 if layout else None)
+
+
+@pytest.mark.slow
+def test_dsa_indexer_nvfp4_interleaved_full_4096x64(hq):
+    seed = S.SEEDS["dsa_indexer"]
+    pe = S.normal_bf16(seed, (4096, 64, 64))
+    nope = S.normal_bf16(seed + 100, (4096, 64, 64))
+    _cat4_case(hq, pe, nope, 4096, 64, 128, oracle.TRANSPOSED | hq.HQ_SF_SWIZZLED, ld=4096)
+
+
 @pytest.mark.slow
 def test_dsa_indexer_nvfp4_full_4096x64(hq):
     seed = S.SEEDS["dsa_indexer"]
@@ -164,6 +200,20 @@ def _k128_case(hq, mode, x, M, K_out):
 def test_k128_bf16_ragged(hq, M, K):
     x = S.with_outliers_bf16(S.normal_bf16(301 + M, (M, K)), 302, p=0.01)
     _k128_case(hq, hq.HQ_ACT_NONE_BF16, x, M, K)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_k128_ue8m0_all_modes(hq, mode):
+    M, K = 33, 640
+    if mode == 0:
+        x = S.with_outliers_bf16(S.normal_bf16(341, (M, K)), 342, p=0.01, factor=1e4)
+    elif mode == 1:
+        x = S.normal_f32(343, (M, K), std=3.0)
+        x[0, :4] = [0.0, -0.0, 1e-30, 448.0]
+        x[1] = 0.0
+    else:
+        x = S.normal_f32(344, (M, 2 * K), std=2 ** 0.5)
+    _k128_case(hq, mode | hq.HQ_FP8_UE8M0, x, M, K)
 
 
 @pytest.mark.parametrize("M,K", [(1, 128), (7, 640), (65, 256)])

@@ -83,7 +83,7 @@ def test_host_entry_matches_oracle(hq):
                      "col codes")
 
 
-@pytest.mark.parametrize("flags", [1, 2, 3 | 4, 3 | 8, 1 | 4])
+@pytest.mark.parametrize("flags", [1, 2, 3 | 4, 3 | 8, 1 | 4, 3 | 128])
 def test_host_entry_flags(hq, flags):
     splits = [128, 256, 0, 128]
     x = _case(621, 256, splits)

@@ -294,7 +294,29 @@ def _run_sr(hq, x, splits, mask, flags, seed, offset):
     return {k: v.cpu().numpy() for k, v in out.items()}
 
 
-@pytest.mark.parametrize("flags", [3 | 32 | 64, 1 | 32, 2 | 64, 3 | 64, 1 | 4 | 32, 3 | 4 | 32 | 64 | 8])
+@pytest.mark.parametrize("flags", [3 | 128, 1 | 4 | 128, 2 | 128, 3 | 8 | 128, 7 | 128])
+def test_interleaved_block_scales(hq, flags):
+    """row_sf and every section's col_sf block in the interleaved 128 x 4 tiles."""
+    splits = [128, 0, 384, 256]
+    x = _case(611, 512, splits)
+    mask = 0x5A3C
+    got, _ = _run(hq, x, splits, mask, flags)
+    _check(got, oracle.group_rht_quant(x, splits, mask, flags & ~8), x, splits, mask, flags & ~8)
+
+
+@pytest.mark.slow
+def test_interleaved_block_scales_grouped_moe_16384x7168(hq):
+    seed = S.SEEDS["grouped_moe"]
+    x = S.normal_bf16(seed, (16384, 7168))
+    splits = S.moe_splits(seed)
+    mask = S.sign_mask16(seed)
+    flags = 3 | hq.HQ_SF_SWIZZLED
+    got, _ = _run(hq, x, splits, mask, flags)
+    _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
+
+
+@pytest.mark.parametrize("flags", [3 | 32 | 64, 1 | 32, 2 | 64, 3 | 64, 1 | 4 | 32, 3 | 4 | 32 | 64 | 8,
+                                   3 | 32 | 64 | 128])
 def test_stochastic_rounding_matches_oracle(hq, flags):
     """Stochastic rounding is decided by integer comparisons of exact values,
     so the codes must be bit-identical to the oracle's."""
@@ -302,7 +324,7 @@ def test_stochastic_rounding_matches_oracle(hq, flags):
     x = _case(501, 384, splits)
     mask, seed, offset = 0x6B2D, 0x0123456789ABCDEF, 16 * 12345
     got = _run_sr(hq, x, splits, mask, flags, seed, offset)
-    base = flags & (1 | 2 | 4 | 32 | 64)
+    base = flags & (1 | 2 | 4 | 32 | 64 | 128)
     want = oracle.group_rht_quant(x, splits, mask, base, seed=seed, offset=offset)
     for k in want:
         assert_bits_equal(got[k], want[k], k)
