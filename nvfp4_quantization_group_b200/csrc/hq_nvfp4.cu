@@ -557,7 +557,7 @@ __device__ __forceinline__ uint32_t nv_producer(const NvParams& p, NvShared& sh,
 // RowRht: the rowwise blocks are rotated along K before their amax and cast.
 // SR: the codes of the directions HQ_ROW_SR / HQ_COL_SR select round
 // stochastically (one Philox block per 16-element block).
-template <bool RowRht, bool SR>
+template <bool RowRht, bool SR, bool Swz>
 __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, const uint8_t* tiles, int w,
                                             int lane) {
     uint32_t* const err = p.ws + 2;
@@ -709,7 +709,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
         } else if (!(h.flags & H_GAVE_UP)) {
             // ===================================================== cast tile
             uint8_t* const rc_base = p.row_codes + (uint64_t)h.row0 * K2 + (uint32_t)h.col0 / 2u;
-            const bool swz = p.flags & HQ_SF_SWIZZLED;
+            constexpr bool swz = Swz;
             // row scales: the plain [M, K/16] rows, or the tile's 1 KB of interleaved tiles
             uint8_t* const rs_base = swz ? p.row_sf + (((uint64_t)h.row0 >> 7) * (K16 >> 2) + ((uint32_t)h.col0 >> 6)) * 512u
                                          : p.row_sf + (uint64_t)h.row0 * K16 + (uint32_t)h.col0 / 16u;
@@ -857,7 +857,7 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
 }  // namespace
 
-template <bool RowRht, bool SR>
+template <bool RowRht, bool SR, bool Swz>
 __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel(const __grid_constant__ NvParams p) {
     extern __shared__ __align__(1024) uint8_t nv_smem_raw[];
     uint8_t* const nv_smem = nv_smem_raw + ((1024u - (smem_u32(nv_smem_raw) & 1023u)) & 1023u);
@@ -905,7 +905,7 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
             mbar_wait_bounded(&sh.full[st], last_use & 1u, MBAR_LIMIT);
         }
     } else {
-        nv_consumer<RowRht, SR>(p, sh, nv_smem, warp, lane);
+        nv_consumer<RowRht, SR, Swz>(p, sh, nv_smem, warp, lane);
     }
 
     // ---- the last CTA to leave publishes the section scales and resets the
@@ -943,13 +943,17 @@ __global__ void __launch_bounds__(NV_THREADS, NV_CTAS_PER_SM) nvfp4_group_kernel
     }
 }
 
+// The instances, indexed by HQ_ROW_RHT | SR << 1 | interleaved scales << 2.
+static void (*const nv_kernels[8])(NvParams) = {
+    nvfp4_group_kernel<false, false, false>, nvfp4_group_kernel<true, false, false>,
+    nvfp4_group_kernel<false, true, false>,  nvfp4_group_kernel<true, true, false>,
+    nvfp4_group_kernel<false, false, true>,  nvfp4_group_kernel<true, false, true>,
+    nvfp4_group_kernel<false, true, true>,   nvfp4_group_kernel<true, true, true>};
+
 int nvfp4_blocks_per_sm() {
-    // both variants: the grid is sized for the one with fewer resident CTAs
-    // every variant: the grid is sized for the one with fewest resident CTAs
-    void (*const kernels[4])(NvParams) = {nvfp4_group_kernel<false, false>, nvfp4_group_kernel<true, false>,
-                                          nvfp4_group_kernel<false, true>, nvfp4_group_kernel<true, true>};
+    // every instance: the grid is sized for the one with fewest resident CTAs
     int n = 1 << 30;
-    for (auto* k : kernels) {
+    for (auto* k : nv_kernels) {
         int m = 0;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, NV_DYN_SMEM);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, k, NV_THREADS, NV_DYN_SMEM);
@@ -966,13 +970,8 @@ int nvfp4_tiles_in_flight_per_cta() { return NST + 2; }
 int nvfp4_tiles_per_claim() { return CLAIM; }
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
-    const bool rot = p.flags & HQ_ROW_RHT, sr = p.flags & (HQ_ROW_SR | HQ_COL_SR);
-    if (sr) {
-        if (rot) nvfp4_group_kernel<true, true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
-        else nvfp4_group_kernel<false, true><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
-    } else {
-        if (rot) nvfp4_group_kernel<true, false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
-        else nvfp4_group_kernel<false, false><<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
-    }
+    const int v = ((p.flags & HQ_ROW_RHT) ? 1 : 0) | ((p.flags & (HQ_ROW_SR | HQ_COL_SR)) ? 2 : 0) |
+                  ((p.flags & HQ_SF_SWIZZLED) ? 4 : 0);
+    nv_kernels[v]<<<grid, NV_THREADS, NV_DYN_SMEM, st>>>(p);
 }
 }  // namespace hq
