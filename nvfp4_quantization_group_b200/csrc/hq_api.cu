@@ -18,7 +18,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     int sms = 0;
     int nv_blocks_per_sm = 0;
-    int cat_blocks_per_sm = 0;
+    int cat_blocks_per_sm[2] = {0, 0};  // FP8, FP4 DSA kernels
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -32,7 +32,8 @@ const DeviceInfo* device_info() {
         DeviceInfo d;
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         d.nv_blocks_per_sm = nvfp4_blocks_per_sm();
-        d.cat_blocks_per_sm = cat_rotate_blocks_per_sm();
+        d.cat_blocks_per_sm[0] = cat_rotate_blocks_per_sm(false);
+        d.cat_blocks_per_sm[1] = cat_rotate_blocks_per_sm(true);
         g_dev[dev] = d;
     });
     const DeviceInfo* d = &g_dev[dev];
@@ -510,14 +511,14 @@ static hq_status cat_rotate(const void* a, int64_t a_row_stride, int a_width, co
     p.scale_ld = scale_ld;
     p.ue8m0 = !fp4 && fmt;
     p.sf_swizzle = fp4 && fmt;
-    p.wide = a_width % 16 == 0 && b_width % 16 == 0 && a_row_stride % 16 == 0 && b_row_stride % 16 == 0 &&
-             (reinterpret_cast<uintptr_t>(a) & 31u) == 0 && (b_width == 0 || (reinterpret_cast<uintptr_t>(b) & 31u) == 0);
+    p.wide32 = a_width % 32 == 0 && b_width % 32 == 0 && a_row_stride % 16 == 0 && b_row_stride % 16 == 0 &&
+               (reinterpret_cast<uintptr_t>(a) & 31u) == 0 && (b_width == 0 || (reinterpret_cast<uintptr_t>(b) & 31u) == 0);
     p.ntiles = cat_rotate_tiles(p);
     if (p.nvec >= ((int64_t)1 << 31) || p.ntiles >= ((int64_t)1 << 31)) return HQ_ERR_SHAPE;
     p.g_magic = 0xFFFFFFFFu / (uint32_t)G;
     p.gt_magic = 0xFFFFFFFFu / (uint32_t)cat_rotate_group_tiles(G);
     const int64_t tiles = p.ntiles;
-    const int64_t cap = (int64_t)dev->sms * (dev->cat_blocks_per_sm > 0 ? dev->cat_blocks_per_sm : 1);
+    const int64_t cap = (int64_t)dev->sms * dev->cat_blocks_per_sm[fp4 ? 1 : 0];
     const int grid = (int)(tiles < cap ? tiles : cap);
     launch_cat_rotate(p, grid, (cudaStream_t)stream, fp4);
     return launch_status();

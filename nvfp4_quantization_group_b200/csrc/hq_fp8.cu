@@ -1,12 +1,12 @@
 // hq_fp8.cu -- FP8 E4M3 group quantizers for sm_100a, and the FP4 variant
 // of the DSA indexer prep.
 //
-//  * cat_rotate_kernel<false>: DSA indexer prep (TensorRT-LLM PR #15158, code
-//    flow "torch.cat -> rotate_activation -> fp8_quantize_1x128"): concat of
-//    the pe and nope parts of each (token, head) vector, 128-point Sylvester
-//    Hadamard rotation scaled by 1/sqrt(128), then one E4M3 group of 128
-//    with the scale rule of onnxruntime PR #33644.
-//  * cat_rotate_kernel<true>: the same concat and rotation, then NVFP4 per
+//  * cat_rotate4_kernel<false>: DSA indexer prep (TensorRT-LLM PR #15158,
+//    code flow "torch.cat -> rotate_activation -> fp8_quantize_1x128"):
+//    concat of the pe and nope parts of each (token, head) vector, 128-point
+//    Sylvester Hadamard rotation scaled by 1/sqrt(128), then one E4M3 group of
+//    128 with the scale rule of onnxruntime PR #33644.
+//  * cat_rotate4_kernel<true>: the same concat and rotation, then NVFP4 per
 //    vector (the FP4 path the same PR names as lacking the rotation): the
 //    vector's amax gives its global encode scale, each 16-element block an
 //    E4M3 scale and E2M1 codes, as in the grouped NVFP4 cast.
@@ -15,8 +15,10 @@
 //    SwiGLU product SiLU(gate) * up.
 //  * convert_kernel: element-wise E4M3 / E2M1 codec.
 //
-// Both quantizers are HBM-bound streams: every input byte is read once with
-// coalesced 16-byte loads and every output byte written once.
+// Both quantizers stream: every input byte is read once with coalesced 16- or
+// 32-byte loads and every output byte written once (the lanes of one store
+// instruction cover whole 32-byte sectors, or halves of them for the FP4
+// DSA codes).
 #include "hq_internal.h"
 
 namespace hq {
@@ -58,39 +60,15 @@ __device__ __forceinline__ uint2 quant8(const f2 (&ny)[4], float s) {
     return quant8_neg(ny, pack2(d.b, d.b), pack2(d.nr, d.nr));
 }
 
-// ------------------------------------------------ cat -> H128 -> FP8 1x128
-// Eight threads share one 128-vector, 16 elements each; a CTA of 256 threads
-// takes a tile of 32 vectors.  The butterfly runs in two halves:
-//  * thread j loads elements 16j..16j+15 (two 16-byte loads, from the pe or
-//    the nope part) and runs stages 1, 2, 4, 8 on them; stage 1 takes the
-//    BF16 pair straight from the load word (mixed-precision add / FMA, one
-//    rounding each, as FP32 additions of the widened values);
-//  * the 8 threads exchange values through shared memory (within the warp,
-//    no CTA barrier) so that thread j then holds elements 16s + 2j and
-//    16s + 2j + 1 for s = 0..7, and runs stages 16, 32, 64 on them.
-// The 8 threads then reduce the amax with 3 shuffles, quantize their 16
-// values, and exchange the codes through shared memory once more so that
-// each writes 16 contiguous bytes.  Tiles are 32 consecutive vectors, or, for
-// transposed scales, 32 consecutive rows of one group (the 32 scales are then
-// contiguous).  The next tile's loads are issued before the current tile is
-// computed.
-constexpr int CAT_THREADS = 256;
+// ------------------------------------------- cat -> H128 -> FP8 / NVFP4: tiles
+// A tile is 32 consecutive vectors, or, for transposed scales, CAT_TT
+// consecutive rows x CAT_TG groups: slot k = (k / CAT_TT) groups on,
+// (k % CAT_TT) rows on, so each group's CAT_TT scales are contiguous;
+// consecutive tiles walk the groups of a row block.
 constexpr int CAT_VEC = 32;  // vectors per tile
-
-struct CatShared {
-    float2 t[CAT_VEC][72];       // 64 pairs of one vector + 8 of padding (bank spread)
-    uint32_t codes[CAT_VEC][36];  // 128 code bytes of one vector + 16 of padding
-};
-
 #ifndef HQ_CAT_TT
 #define HQ_CAT_TT 8
 #endif
-#ifndef HQ_CAT_MINB
-#define HQ_CAT_MINB 3
-#endif
-// Transposed scales: a tile is CAT_TT consecutive rows x CAT_TG groups, slot
-// k = (k / CAT_TT) groups on, (k % CAT_TT) rows on, so each group's CAT_TT
-// scales are contiguous; consecutive tiles walk the groups of a row block.
 constexpr int CAT_TT = HQ_CAT_TT, CAT_TG = CAT_VEC / CAT_TT;
 
 // x / d and x % d for 32-bit x by multiply-high with m = floor((2^32 - 1) / d)
@@ -129,61 +107,98 @@ __device__ __forceinline__ CatVec cat_vector(const CatRotateParams& p, uint32_t 
     return r;
 }
 
-// Where thread j's 16 elements of every vector come from in the wide layout
-// (whole segments in a or in b): the same input for all vectors, so the
-// choice and its strides are made once per thread.
+// Base and strides of one thread's elements in one input.
 struct CatSrc {
-    const uint16_t* base;  // element 16j of vector (0, 0)
+    const uint16_t* base;  // thread j's first element of vector (0, 0)
     int64_t tstride;       // per row t
     int gwidth;            // per group g
 };
-__device__ __forceinline__ CatSrc cat_src(const CatRotateParams& p, int j) {
-    const int a_chunks = p.a_width / 8;
+
+// ------------------------------------------------ cat -> H128 -> FP8 / NVFP4
+// Four threads share one 128-vector, 32 elements each; a CTA of 128 threads
+// takes a tile of 32 vectors.  The next tile's loads are issued before the
+// current tile is computed.
+//  * thread j loads elements 32j..32j+31 (two 32-byte loads when the pe/nope
+//    split is a multiple of 32, else four 16-byte chunks, each from pe or
+//    nope) and runs butterfly stages 1, 2, 4, 8, 16 on them; stage 1 takes
+//    the BF16 pair straight from the load word (mixed-precision add / FMA,
+//    one rounding each, as FP32 additions of the widened values);
+//  * one exchange through shared memory (within the warp) gives thread j the
+//    elements 32m + 8j .. 32m + 8j + 7 for m = 0..3, on which it runs stages
+//    32 and 64;
+//  * the 4 threads reduce the amax with 2 shuffles and quantize their 32
+//    values; for each m the codes of elements 32m + 8j .. 32m + 8j + 7 are 8
+//    contiguous output bytes (FP8), stored without a second exchange.
+//  * NVFP4 (FP4): the 16-element block 2m + j/2 is split over threads j and
+//    j ^ 1 (8 elements each); one shuffle gives its amax, both threads form
+//    its scale and encode factor, and each stores its 4 bytes of codes.
+// The stages run in ascending order.
+constexpr int CAT4_THREADS = 128;
+// resident CTAs the register allocation is capped for (FP8: 120 registers,
+// FP4: 93; measured best of 3 to 6)
+constexpr int CAT4_MINB_FP8 = 4, CAT4_MINB_FP4 = 5;
+
+struct Cat4Shared {
+    // per vector: thread m's 32 floats at float4 8m .. 8m + 7, its chunk q
+    // (elements 32m + 4q .. 4q + 3) at 8m + ((q + 2m) & 7); 33 float4 per
+    // vector.  A quarter-warp (2 vectors x 4 threads) then hits 8 different
+    // 4-bank groups in both the writes and the reads.
+    float4 t[CAT_VEC][33];
+};
+
+// Where thread j's 32 elements of every vector come from when they lie in
+// one input (wide32): its base and strides, chosen once.
+__device__ __forceinline__ CatSrc cat4_src(const CatRotateParams& p, int j) {
     CatSrc s;
-    if (2 * j < a_chunks) {
-        s.base = p.a + j * 16;
+    if (32 * j < p.a_width) {
+        s.base = p.a + 32 * j;
         s.tstride = p.a_row_stride;
         s.gwidth = p.a_width;
     } else {
-        s.base = p.b + (2 * j - a_chunks) * 8;
+        s.base = p.b + (32 * j - p.a_width);
         s.tstride = p.b_row_stride;
         s.gwidth = p.b_width;
     }
     return s;
 }
 
-// The two 16-byte chunks (elements 16j..16j+15) of vector (t, g).
-__device__ __forceinline__ void cat_load(const CatRotateParams& p, const CatSrc& src, CatVec cv, int j, uint4& c0,
-                                         uint4& c1) {
-    c0 = c1 = make_uint4(0u, 0u, 0u, 0u);
+// Elements 32j..32j+31 of vector (t, g) as 16 BF16 pairs (zeros past the end).
+__device__ __forceinline__ void cat4_load(const CatRotateParams& p, const CatSrc& src, CatVec cv, int j,
+                                          uint4 (&c)[4]) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) c[h] = make_uint4(0u, 0u, 0u, 0u);
     if (cv.t < 0) return;
     const int64_t t = cv.t;
     const int g = cv.g;
-    const int a_chunks = p.a_width / 8;
-    if (p.wide) {
-        ld_nc_v8(src.base + (t * src.tstride + (int64_t)g * src.gwidth), c0, c1);
+    if (p.wide32) {
+        const uint16_t* s = src.base + (t * src.tstride + (int64_t)g * src.gwidth);
+        ld_nc_v8(s, c[0], c[1]);
+        ld_nc_v8(s + 16, c[2], c[3]);
         return;
     }
+    const int a_chunks = p.a_width / 8;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int c = 2 * j + h;
-        const uint16_t* src = c < a_chunks
-            ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + c * 8
-            : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (c - a_chunks) * 8;
-        (h ? c1 : c0) = ld_nc_v4(src);
+    for (int h = 0; h < 4; ++h) {
+        const int ch = 4 * j + h;
+        const uint16_t* s = ch < a_chunks
+            ? p.a + t * p.a_row_stride + (int64_t)g * p.a_width + ch * 8
+            : p.b + t * p.b_row_stride + (int64_t)g * p.b_width + (ch - a_chunks) * 8;
+        c[h] = ld_nc_v4(s);
     }
 }
 
 template <bool FP4>
-__global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(CatRotateParams p) {
-    __shared__ CatShared sh;
+__global__ void __launch_bounds__(CAT4_THREADS, FP4 ? CAT4_MINB_FP4 : CAT4_MINB_FP8)
+    cat_rotate4_kernel(CatRotateParams p) {
+    __shared__ Cat4Shared sh;
     __shared__ float2 vr[FP4 ? 128 : 1];  // FP4: per E4M3 code {value, -RN(1 / value)}
-    const int tid = threadIdx.x, k = tid >> 3, j = tid & 7;
+    const int tid = threadIdx.x, k = tid >> 2, j = tid & 3;
     if constexpr (FP4) {
+        static_assert(CAT4_THREADS >= 128, "one thread per code");
         if (tid < 128) {
-            const bool z = tid == 0 || tid == 127;
-            const float v = z ? 0.0f : e4m3_value((uint32_t)tid);
-            vr[tid] = make_float2(v, z ? -0.0f : -__frcp_rn(v));
+            const bool zc = tid == 0 || tid == 127;
+            const float v = zc ? 0.0f : e4m3_value((uint32_t)tid);
+            vr[tid] = make_float2(v, zc ? -0.0f : -__frcp_rn(v));
         }
         __syncthreads();
     }
@@ -193,31 +208,33 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
     const CatVec none{-1, 0};
     uint32_t tile = blockIdx.x;
     const uint32_t ntiles = (uint32_t)p.ntiles;
-    uint4 n0, n1;  // the next tile's chunks
-    const CatSrc src = cat_src(p, j);
+    uint4 nc[4];  // the next tile's load words
+    const CatSrc src = cat4_src(p, j);
     CatVec nv = tile < ntiles ? cat_vector(p, tile, k) : none;
-    cat_load(p, src, nv, j, n0, n1);
+    cat4_load(p, src, nv, j, nc);
+    float4* const row = sh.t[k];
     for (; tile < ntiles; tile += gridDim.x) {
         const CatVec cv = nv;
-        const uint32_t w[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+        const uint32_t w[16] = {nc[0].x, nc[0].y, nc[0].z, nc[0].w, nc[1].x, nc[1].y, nc[1].z, nc[1].w,
+                                nc[2].x, nc[2].y, nc[2].z, nc[2].w, nc[3].x, nc[3].y, nc[3].z, nc[3].w};
         const uint32_t nt = tile + gridDim.x;
         nv = nt < ntiles ? cat_vector(p, nt, k) : none;
-        cat_load(p, src, nv, j, n0, n1);
+        cat4_load(p, src, nv, j, nc);
 
-        // ---- elements 16j..16j+15 as 8 pairs (2i, 2i+1) of this segment
-        f2 y[8];
+        // ---- elements 32j + 2i, 32j + 2i + 1
+        f2 y[16];
         if (p.rotate) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 16; ++i) {
                 bf16_t lo, hi;
                 split_bf16x2(w[i], lo, hi);
                 const float x0 = bf16_lo(w[i]);
                 y[i] = pack2(add_bf16(hi, x0), fma_bf16(hi, minus_one, x0));  // stage 1
             }
 #pragma unroll
-            for (int h = 1; h < 8; h <<= 1) {  // stages 2, 4, 8
+            for (int h = 1; h < 16; h <<= 1) {  // stages 2, 4, 8, 16
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     if ((i & h) == 0) {
                         const f2 a = y[i], b = y[i + h];
                         y[i] = add2(a, b);
@@ -227,36 +244,40 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = pack2(bf16_lo(w[i]), bf16_hi(w[i]));
+            for (int i = 0; i < 16; ++i) y[i] = pack2(bf16_lo(w[i]), bf16_hi(w[i]));
         }
-        // ---- exchange: thread j now takes pair j of every segment s
-        // (16-byte piece c of segment s is stored at position (c + s/2) & 3 of
-        // the segment's 64 bytes: the 8 lanes of a vector then hit 8
-        // different bank groups when writing)
-        float4* row = reinterpret_cast<float4*>(&sh.t[k][8 * j]);
+        // ---- exchange: thread j now takes elements 32m + 8j .. 32m + 8j + 7
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int q = 0; q < 8; ++q) {
             float a0, a1, b0, b1;
-            unpack2(y[2 * c], a0, a1);
-            unpack2(y[2 * c + 1], b0, b1);
-            row[(c + (j >> 1)) & 3] = make_float4(a0, a1, b0, b1);
+            unpack2(y[2 * q], a0, a1);
+            unpack2(y[2 * q + 1], b0, b1);
+            row[8 * j + ((q + 2 * j) & 7)] = make_float4(a0, a1, b0, b1);
         }
         __syncwarp();
-        f2 z[8];
+        f2 z[4][4];  // z[m][l]: elements 32m + 8j + 2l, 32m + 8j + 2l + 1
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            const float2 e = sh.t[k][8 * s + 2 * (((j >> 1) + (s >> 1)) & 3) + (j & 1)];
-            z[s] = pack2(e.x, e.y);
+        for (int m = 0; m < 4; ++m) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 e = row[8 * m + ((2 * j + h + 2 * m) & 7)];
+                z[m][2 * h] = pack2(e.x, e.y);
+                z[m][2 * h + 1] = pack2(e.z, e.w);
+            }
         }
+        __syncwarp();  // every read is done before the next tile's writes
         if (p.rotate) {
 #pragma unroll
-            for (int h = 1; h < 8; h <<= 1) {  // stages 16, 32, 64
+            for (int h = 1; h < 4; h <<= 1) {  // stages 32 (m, m + 1) and 64 (m, m + 2)
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    if ((s & h) == 0) {
-                        const f2 a = z[s], b = z[s + h];
-                        z[s] = add2(a, b);
-                        z[s + h] = sub2(a, b);
+                for (int m = 0; m < 4; ++m) {
+                    if ((m & h) == 0) {
+#pragma unroll
+                        for (int l = 0; l < 4; ++l) {
+                            const f2 a = z[m][l], b = z[m + h][l];
+                            z[m][l] = add2(a, b);
+                            z[m + h][l] = sub2(a, b);
+                        }
                     }
                 }
             }
@@ -264,92 +285,108 @@ __global__ void __launch_bounds__(CAT_THREADS, HQ_CAT_MINB) cat_rotate_kernel(Ca
         const f2 nc2 = pack2(p.rotate ? neg_c128 : -1.0f, p.rotate ? neg_c128 : -1.0f);
         float amax = 0.0f;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            z[s] = mul2(z[s], nc2);  // -y (exact negation when not rotating)
-            float a, b;
-            unpack2(z[s], a, b);
-            amax = absmax3(amax, a, b);
+        for (int m = 0; m < 4; ++m) {
+#pragma unroll
+            for (int l = 0; l < 4; ++l) {
+                z[m][l] = mul2(z[m][l], nc2);  // -y (exact negation when not rotating)
+                float a, b;
+                unpack2(z[m][l], a, b);
+                amax = absmax3(amax, a, b);
+            }
         }
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 4));
         if constexpr (FP4) {
-            // ---- NVFP4: back to one 16-element block per thread (pair j of
-            // segment s at position (j + s) & 7 of the segment: both sides
-            // free of bank conflicts), then block scale and codes
             const float S = global_encode(amax);
-            __syncwarp();  // the first exchange is read
+            const bool slow = slow_scale(S);
+            uint32_t codes[4], sfs[4];
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                float a, b;
-                unpack2(z[s], a, b);
-                sh.t[k][8 * s + ((j + s) & 7)] = make_float2(-a, -b);  // y = -z exactly
+            for (int m = 0; m < 4; ++m) {
+                float yv[8];  // y = -z exactly
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    float a, b;
+                    unpack2(z[m][l], a, b);
+                    yv[2 * l] = -a;
+                    yv[2 * l + 1] = -b;
+                }
+                // the block's amax: this thread's 8 values and its partner's
+                // (max is exact and skips a NaN, as over the 16 at once)
+                const float a8 = max3(max3(fabsf(yv[0]), fabsf(yv[1]), fabsf(yv[2])),
+                                      max3(fabsf(yv[3]), fabsf(yv[4]), fabsf(yv[5])),
+                                      max3(fabsf(yv[6]), fabsf(yv[7]), 0.0f));
+                const float ab = fmaxf(a8, __shfl_xor_sync(0xFFFFFFFFu, a8, 1));
+                const uint32_t sf = block_sf(ab, S);
+                const float enc = block_enc(vr, sf, S, slow);
+                const f2 e2 = pack2(enc, enc);
+                float qv[8];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) unpack2(mul2(pack2(yv[2 * l], yv[2 * l + 1]), e2), qv[2 * l], qv[2 * l + 1]);
+                codes[m] = e2m1x8(qv[0], qv[1], qv[2], qv[3], qv[4], qv[5], qv[6], qv[7]);
+                sfs[m] = sf;
             }
-            __syncwarp();
-            float y[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float2 e = sh.t[k][8 * j + ((i + j) & 7)];
-                y[2 * i] = e.x;
-                y[2 * i + 1] = e.y;
-            }
-            const uint32_t sf = block_sf(absmax16(y), S);
-            const float enc = block_enc(vr, sf, S, slow_scale(S));
-            const f2 e2 = pack2(enc, enc);
-            float q[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) unpack2(mul2(pack2(y[2 * i], y[2 * i + 1]), e2), q[2 * i], q[2 * i + 1]);
             if (cv.t >= 0) {
                 const int64_t v = (int64_t)cv.t * p.G + cv.g;
-                *reinterpret_cast<uint2*>(p.out + v * 64 + 8 * j) =
-                    make_uint2(e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]),
-                               e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]));
-                p.sf[p.sf_swizzle ? sf_swizzled((uint64_t)cv.t, (uint64_t)cv.g * 8u + (uint64_t)j, (uint64_t)p.G * 8u)
-                                  : (uint64_t)v * 8u + (uint64_t)j] = (uint8_t)sf;
+                // elements 32m + 8j .. 32m + 8j + 7: bytes 16m + 4j .. 16m + 4j + 3
+                uint8_t* const o = p.out + v * 64 + 4 * j;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) *reinterpret_cast<uint32_t*>(o + 16 * m) = codes[m];
+                if ((j & 1) == 0) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint64_t blk = (uint64_t)(2 * m + (j >> 1));
+                        p.sf[p.sf_swizzle ? sf_swizzled((uint64_t)cv.t, (uint64_t)cv.g * 8u + blk, (uint64_t)p.G * 8u)
+                                          : (uint64_t)v * 8u + blk] = (uint8_t)sfs[m];
+                    }
+                }
                 if (j == 0) {
                     const int64_t si = p.scale_layout == 0 ? v : (int64_t)cv.g * p.scale_ld + cv.t;
                     p.scales[si] = __fdiv_rn(1.0f, S);
                     if (p.amax) p.amax[si] = amax;
                 }
             }
-            __syncwarp();  // the exchange buffer is reused by the next tile
             continue;
         }
         const float sc = p.ue8m0 ? ue8m0_up(fp8_group_scale(amax)) : fp8_group_scale(amax);
-        // ---- codes of elements 16s + 2j, 16s + 2j + 1
-        uint32_t q[8];
+        uint2 q[4];
         if (!isinf(sc)) {
             const Recip d = make_recip(sc);
             const f2 b2 = pack2(d.b, d.b), nr2 = pack2(d.nr, d.nr);
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                float a, b;
-                unpack2(div2_rn_neg(z[s], b2, nr2), a, b);
-                q[s] = e4m3x2(a, b);
+            for (int m = 0; m < 4; ++m) {
+                uint32_t c[4];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    float a, b;
+                    unpack2(div2_rn_neg(z[m][l], b2, nr2), a, b);
+                    c[l] = e4m3x2(a, b);
+                }
+                q[m] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
             }
         } else {  // an infinite input: plain IEEE division
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                float a, b;
-                unpack2(z[s], a, b);
-                q[s] = e4m3x2(__fdiv_rn(-a, sc), __fdiv_rn(-b, sc));
+            for (int m = 0; m < 4; ++m) {
+                uint32_t c[4];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    float a, b;
+                    unpack2(z[m][l], a, b);
+                    c[l] = e4m3x2(__fdiv_rn(-a, sc), __fdiv_rn(-b, sc));
+                }
+                q[m] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
             }
         }
-        uint16_t* cb = reinterpret_cast<uint16_t*>(sh.codes[k]);
-#pragma unroll
-        for (int s = 0; s < 8; ++s) cb[8 * s + j] = (uint16_t)q[s];
-        __syncwarp();
         if (cv.t >= 0) {
             const int64_t v = (int64_t)cv.t * p.G + cv.g;
-            const uint4 out = *reinterpret_cast<const uint4*>(&sh.codes[k][4 * j]);
-            *reinterpret_cast<uint4*>(p.out + v * 128 + 16 * j) = out;
+            uint8_t* const o = p.out + v * 128 + 8 * j;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) *reinterpret_cast<uint2*>(o + 32 * m) = q[m];
             if (j == 0) {
                 const int64_t si = p.scale_layout == 0 ? v : (int64_t)cv.g * p.scale_ld + cv.t;
                 p.scales[si] = sc;
                 if (p.amax) p.amax[si] = amax;
             }
         }
-        __syncwarp();  // the exchange buffers are reused by the next tile
     }
 }
 
@@ -521,20 +558,18 @@ int64_t cat_rotate_tiles(const CatRotateParams& p) {
                                : ((p.G + CAT_TG - 1) / CAT_TG) * ((p.M + CAT_TT - 1) / CAT_TT);
 }
 
-int cat_rotate_blocks_per_sm() {
-    // both variants: the grid is sized for the one with fewer resident CTAs
-    int n0 = 0, n1 = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n0, cat_rotate_kernel<false>, CAT_THREADS, 0);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n1, cat_rotate_kernel<true>, CAT_THREADS, 0);
-    const int n = n0 < n1 ? n0 : n1;
+int cat_rotate_blocks_per_sm(bool fp4) {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fp4 ? cat_rotate4_kernel<true> : cat_rotate4_kernel<false>,
+                                                  CAT4_THREADS, 0);
     return n > 0 ? n : 1;
 }
 
 void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st, bool fp4) {
     if (fp4)
-        cat_rotate_kernel<true><<<grid, CAT_THREADS, 0, st>>>(p);
+        cat_rotate4_kernel<true><<<grid, CAT4_THREADS, 0, st>>>(p);
     else
-        cat_rotate_kernel<false><<<grid, CAT_THREADS, 0, st>>>(p);
+        cat_rotate4_kernel<false><<<grid, CAT4_THREADS, 0, st>>>(p);
 }
 
 template <bool AMAX>

@@ -22,7 +22,7 @@ struct CatRotateParams {
     int64_t ntiles;  // tiles of 32 vectors (see cat_rotate_tiles)
     uint32_t g_magic;      // floor((2^32 - 1) / G): v / G by multiply-high
     uint32_t gt_magic;     // the same for the group tiles of the transposed layout
-    int wide;              // 16-element segments never straddle a and b, 32-byte aligned: 32-byte loads
+    int wide32;            // 32-element quarters never straddle a and b, 32-byte aligned: 32-byte loads
     int G;
     int rotate;    // 1: H128 / sqrt(128); 0: none
     uint8_t* out;     // FP8: codes [M, G*128]; FP4: E2M1 codes [M, G*64]
@@ -49,7 +49,7 @@ struct K128Params {
 constexpr int K128_THREADS = 256;   // 8 warps, two K128 groups per warp step
 constexpr int K128_UNROLL = 4;      // warp steps with loads in flight
 
-int cat_rotate_blocks_per_sm();
+int cat_rotate_blocks_per_sm(bool fp4);  // resident CTAs of the FP8 / FP4 kernel
 int64_t cat_rotate_tiles(const CatRotateParams& p);
 int cat_rotate_group_tiles(int G);  // group tiles of the transposed-scale layout
 void launch_cat_rotate(const CatRotateParams& p, int grid, cudaStream_t st, bool fp4);

@@ -72,6 +72,21 @@ def test_cat_unequal_widths_and_strided_rows(hq):
     assert_fp8_codes(codes.cpu().numpy(), want_c)
 
 
+@pytest.mark.parametrize("a_width", [8, 40, 96, 120, 128])
+def test_cat_split_widths_fp8_and_nvfp4(hq, a_width):
+    """pe/nope splits whose 32-element quarter vectors straddle the two inputs
+    (8, 40, 120), lie in one of them (96: the 32-byte load path) or have no
+    second input (128); both outputs, both scale layouts."""
+    M, G = 21, 3
+    pe = S.normal_bf16(271 + a_width, (M, G, a_width))
+    nope = None if a_width == 128 else \
+        S.with_outliers_bf16(S.normal_bf16(272 + a_width, (M, G, 128 - a_width)), 273, p=0.02)
+    for layout in (oracle.ROWMAJOR, oracle.TRANSPOSED):
+        ld = M + 3 if layout else None
+        _cat_case(hq, pe, nope, M, G, 128, layout, ld=ld)
+        _cat4_case(hq, pe, nope, M, G, 128, layout, ld=ld)
+
+
 def test_cat_zero_and_constant_vectors(hq):
     M, G = 3, 2
     pe = np.zeros((M, G, 64), dtype=np.uint16)
