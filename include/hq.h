@@ -66,9 +66,14 @@ typedef enum hq_status {
                               interleaved 128 x 4 tiles that block-scaled
                               tcgen05 MMAs read (see below) */
 #define HQ_TWO_PASS 8u     /* schedule: amax pass and cast pass as two launches
-                              instead of one launch in which each section's
-                              cast follows its amax while the rows are still
-                              in L2; results are identical */
+                              (without HQ_ROW_RHT the amax pass is a streaming
+                              kernel of its own) instead of one launch in which
+                              each section's cast follows its amax while the
+                              rows are still in L2.  A call whose only
+                              non-empty section fills the grid at least once,
+                              without HQ_ROW_RHT, takes two launches without
+                              the flag too (its casts wait for the whole amax
+                              pass either way).  Results are identical. */
 
 /* hq_cat_rotate_fp8 scale layouts */
 #define HQ_SCALE_ROWMAJOR 0   /* scale of group (t, g) at scales[t * G + g] */

@@ -19,6 +19,7 @@ struct DeviceInfo {
     int sms = 0;
     int nv_blocks_per_sm = 0;
     int cat_blocks_per_sm[2] = {0, 0};  // FP8, FP4 DSA kernels
+    int amax_blocks_per_sm = 0;
 };
 
 DeviceInfo g_dev[kMaxDevices];
@@ -34,6 +35,7 @@ const DeviceInfo* device_info() {
         d.nv_blocks_per_sm = nvfp4_blocks_per_sm();
         d.cat_blocks_per_sm[0] = cat_rotate_blocks_per_sm(false);
         d.cat_blocks_per_sm[1] = cat_rotate_blocks_per_sm(true);
+        d.amax_blocks_per_sm = nvfp4_amax_blocks_per_sm();
         g_dev[dev] = d;
     });
     const DeviceInfo* d = &g_dev[dev];
@@ -272,7 +274,12 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
         p.reset_counter = 1;
         return launch(p, next);
     }
-    if (!(flags & HQ_TWO_PASS)) {
+    // One non-empty section (a dense tensor): its casts wait for the whole
+    // amax pass in one launch too, and the streaming amax kernel reads faster
+    // than amax tiles do, so two launches unless the section is smaller than
+    // one wave of the grid (then the second launch costs more).
+    const bool one_section = nlive == 1 && !(flags & HQ_ROW_RHT) && tiles_of(live[0]) >= (uint32_t)max_grid;
+    if (!(flags & HQ_TWO_PASS) && !one_section) {
         // One launch.  The cast segment of a section follows its amax segment
         // once `lag` more tiles have been scheduled (the tiles the grid holds
         // in flight), so its amax is normally complete when its first tile is
@@ -302,18 +309,26 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
         p.reset_counter = 1;
         return launch(p, next);
     }
-    // two launches: all amax tiles, then all cast tiles
+    // two launches: all amax tiles, then all cast tiles, the sections in
+    // reverse order (the last rows the amax launch read are still in L2)
     NvParams pa = p, pc = p;
     uint32_t na = 0, nc = 0;
-    for (int k = 0; k < nlive; ++k) {
-        add_seg(pa, live[k], 0, na);
-        add_seg(pc, live[k], 1, nc);
-    }
+    for (int k = 0; k < nlive; ++k) add_seg(pa, live[k], 0, na);
+    for (int k = nlive - 1; k >= 0; --k) add_seg(pc, live[k], 1, nc);
     pa.finalize = 0;
     pa.reset_counter = 1;
     pc.finalize = 1;
     pc.reset_counter = 1;
-    hq_status r = launch(pa, na);
+    hq_status r;
+    if (!(flags & HQ_ROW_RHT)) {
+        // the streaming amax kernel over all tiles (empty sections have none)
+        const uint32_t ntiles = (uint32_t)(M / NV_TILE) * (uint32_t)p.col_tiles;
+        const uint32_t cap = (uint32_t)dev->sms * (uint32_t)dev->amax_blocks_per_sm;
+        if (ntiles > 0) launch_nvfp4_amax(pa, ntiles, (int)(ntiles < cap ? ntiles : cap), st);
+        r = launch_status();
+    } else {
+        r = launch(pa, na);
+    }
     if (r != HQ_OK) return r;
     return launch(pc, nc);
 }

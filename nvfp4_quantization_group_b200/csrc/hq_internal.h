@@ -174,5 +174,9 @@ int nvfp4_blocks_per_sm();
 int nvfp4_tiles_in_flight_per_cta();  // buffers + the claims in flight
 int nvfp4_tiles_per_claim();
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st);
+// The section maxima alone (no row RHT), for the two-pass schedule: leaves
+// the workspace as the amax launch of nvfp4_group_kernel does.
+int nvfp4_amax_blocks_per_sm();
+void launch_nvfp4_amax(const NvParams& p, uint32_t ntiles, int grid, cudaStream_t st);
 
 }  // namespace hq

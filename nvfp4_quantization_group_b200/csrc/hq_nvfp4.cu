@@ -855,6 +855,94 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
     }
 }
 
+// ------------------------------------------------------------ amax kernel
+// The section maxima of the two-pass schedule's first launch, streamed
+// through registers (rowwise output without the row RHT): a CTA of 8 warps
+// takes a 128 x 128 tile (grid-stride, in tile order), warp w its rows
+// 16w..16w+15 and lane l the columns 4l..4l+3 of them: 16 eight-byte loads
+// per lane, each warp load instruction one 256-byte row segment, and the
+// next tile's 16 issued before the current one is computed (2 CTAs of 128
+// registers per SM).  The rowwise maximum is taken on the BF16 magnitudes,
+// the columnwise one over the RHT16 outputs of the lane's two column pairs
+// (the functions of the fused kernel's amax tiles).  A tile's maxima and
+// count are published as the amax tiles publish theirs, so the cast launch
+// that follows finds the same workspace state.  (Measured against it: the
+// same without the prefetch at 2-4 CTAs per SM, up to 11 us slower on the
+// grouped MoE call; a TMA-fed version, one CTA per SM with 6 buffers and 16
+// compute warps, 22 us slower.)
+constexpr int NA_THREADS = 256;
+
+__global__ void __launch_bounds__(NA_THREADS, 2) nvfp4_amax_kernel(const __grid_constant__ NvParams p, uint32_t ntiles) {
+    __shared__ uint32_t acc[2][2];  // [tile parity][rowwise, columnwise] maxima as binary32 bits
+    __shared__ int32_t sec_row0[HQ_MAX_SECTIONS + 1];
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    for (int i = tid; i <= p.S; i += NA_THREADS) sec_row0[i] = p.sec_row0[i];
+    if (tid < 4) acc[tid >> 1][tid & 1] = 0u;
+    bf16_t sg[16];  // sigma_i as BF16 +-1
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sg[i] = ((p.sign_mask >> i) & 1u) ? (bf16_t)0xBF80u : (bf16_t)0x3F80u;
+    const bool do_row = p.flags & HQ_ROWWISE, do_col = p.flags & HQ_COLWISE;
+    uint32_t* const amax_row_ws = p.ws + NV_WS_HEADER;
+    uint32_t* const amax_col_ws = amax_row_ws + p.S;
+    uint32_t* const done_ws = amax_col_ws + p.S;
+    const uint32_t ct = (uint32_t)p.col_tiles;
+    __syncthreads();
+    int s = 0;  // thread 0: section of the current tile (tiles come in increasing order)
+    uint32_t it = 0;
+    uint32_t na[16], nb[16];
+    auto load = [&](uint32_t t) {
+        const uint32_t rt = t / ct, cti = t - rt * ct;
+        const uint16_t* src = p.x + ((int64_t)rt * NV_TILE + 16 * w) * p.K + (int64_t)cti * NV_TILE + 4 * lane;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + i * p.K));
+            na[i] = v.x;
+            nb[i] = v.y;
+        }
+    };
+    if (blockIdx.x < ntiles) load(blockIdx.x);
+    for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+        const uint32_t rt = t / ct;
+        uint32_t wa[16], wb[16];  // row i: columns 4l, 4l + 1 and 4l + 2, 4l + 3
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            wa[i] = na[i];
+            wb[i] = nb[i];
+        }
+        if (t + gridDim.x < ntiles) load(t + gridDim.x);
+        uint32_t mrow = 0u;
+        float mcol = 0.0f;
+        if (do_row) {
+            uint32_t m2 = 0u;  // BF16 pair of running magnitude maxima (a NaN is skipped)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) m2 = hmax_abs(m2, hmax_abs(wa[i], wb[i]));
+            mrow = halves_max_bits(m2);
+        }
+        if (do_col) {
+            mcol = column_rht_absmax(wa, sg, 0.0f);
+            mcol = column_rht_absmax(wb, sg, mcol);
+        }
+        // non-negative binary32 bits order as integers; max |0.25 y| == RN(0.25 max |y|)
+        mrow = __reduce_max_sync(0xFFFFFFFFu, mrow);
+        const uint32_t mc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(__fmul_rn(mcol, 0.25f)));
+        if (lane == 0) {
+            atomicMax(&acc[it & 1u][0], mrow);
+            atomicMax(&acc[it & 1u][1], mc);
+        }
+        __syncthreads();  // (slot it & 1 is next written two tiles on, after the next barrier)
+        if (tid == 0) {
+            while (sec_row0[s + 1] <= (int)(rt * NV_TILE)) ++s;
+            const uint32_t ar = acc[it & 1u][0], ac = acc[it & 1u][1];
+            acc[it & 1u][0] = 0u;
+            acc[it & 1u][1] = 0u;
+            if (do_row) red_max_u32(amax_row_ws + s, ar);
+            if (do_col) red_max_u32(amax_col_ws + s, ac);
+            // release: a producer that sees the count sees the maxima
+            red_release_add_u32(done_ws + s, 1u);
+        }
+    }
+}
+
 }  // namespace
 
 template <bool RowRht, bool SR, bool Swz>
@@ -968,6 +1056,16 @@ int nvfp4_blocks_per_sm() {
 int nvfp4_tiles_in_flight_per_cta() { return NST + 2; }
 
 int nvfp4_tiles_per_claim() { return CLAIM; }
+
+int nvfp4_amax_blocks_per_sm() {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4_amax_kernel, NA_THREADS, 0);
+    return n > 0 ? n : 1;
+}
+
+void launch_nvfp4_amax(const NvParams& p, uint32_t ntiles, int grid, cudaStream_t st) {
+    nvfp4_amax_kernel<<<grid, NA_THREADS, 0, st>>>(p, ntiles);
+}
 
 void launch_nvfp4(const NvParams& p, int grid, cudaStream_t st) {
     const int v = ((p.flags & HQ_ROW_RHT) ? 1 : 0) | ((p.flags & (HQ_ROW_SR | HQ_COL_SR)) ? 2 : 0) |

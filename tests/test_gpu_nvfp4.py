@@ -157,6 +157,37 @@ def test_extreme_magnitudes(hq):
     _check(got, oracle.group_rht_quant(x, splits, 0x8001, 3), x, splits, 0x8001, 3)
 
 
+@pytest.mark.parametrize("flags", [3 | 8, 1 | 8, 2 | 8])
+def test_two_pass_extreme_magnitudes(hq, flags):
+    """The two-launch schedule (its amax pass the streaming amax kernel) on
+    tiny, huge and zero blocks, each direction alone and both."""
+    splits = [128, 0, 128, 128]
+    xf = S.bf16_bits_to_f32(S.normal_bf16(461, (384, 384))).copy()
+    xf[:128] *= np.float32(1e-30)
+    xf[128:256] *= np.float32(1e30)
+    xf[256:, :16] = 0.0
+    xf[300, 40:56] = -0.0
+    x = S.f32_to_bf16_bits(xf)
+    base = flags & ~8
+    got, ws = _run(hq, x, splits, 0x8001, flags)
+    _check(got, oracle.group_rht_quant(x, splits, 0x8001, base), x, splits, 0x8001, base)
+    assert torch.count_nonzero(ws).item() == 0
+
+
+def test_one_large_section_2304x2176(hq):
+    """One non-empty section of 306 tiles, at least one wave of the grid: the
+    library takes two launches (streaming amax, then the casts) without the
+    flag; every output as the oracle, the workspace back at rest."""
+    splits = [0, 2304, 0]
+    x = _case(471, 2176, splits, outliers=0.001)
+    mask = S.sign_mask16(472)
+    ws = hq.new_workspace(len(splits))
+    for flags in (3, 1, 2, 3 | 128, 7):
+        got, ws = _run(hq, x, splits, mask, flags, ws=ws)
+        _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
+        assert torch.count_nonzero(ws).item() == 0
+
+
 @pytest.mark.parametrize("flags", [1 | 4, 1 | 2 | 4, 1 | 2 | 4 | 8])
 def test_row_rht_small_sections(hq, flags):
     """Rowwise blocks rotated along K: both schedules, with and without the
@@ -195,14 +226,15 @@ def test_dense_nvfp4_8192x4096(hq):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("flags", [3, 7])
+@pytest.mark.parametrize("flags", [3, 7, 3 | 8])
 def test_grouped_moe_16384x7168(hq, flags):
     seed = S.SEEDS["grouped_moe"]
     x = S.normal_bf16(seed, (16384, 7168))
     splits = S.moe_splits(seed)
     mask = S.sign_mask16(seed)
     got, _ = _run(hq, x, splits, mask, flags)
-    _check(got, oracle.group_rht_quant(x, splits, mask, flags), x, splits, mask, flags)
+    base = flags & ~8
+    _check(got, oracle.group_rht_quant(x, splits, mask, base), x, splits, mask, base)
 
 
 def _run_given(hq, x, splits, mask, flags, amax_row=None, amax_col=None, ws=None):
