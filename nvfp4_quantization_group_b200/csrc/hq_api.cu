@@ -231,6 +231,7 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
     p.sr_seed = sr_seed;
     p.sr_offset = sr_offset;
     p.col_tiles = (int)(K / NV_TILE);
+    p.done_per_tile = 1;
     int row0 = 0;
     int live[HQ_MAX_SECTIONS];
     int nlive = 0;
@@ -325,6 +326,7 @@ static hq_status group_rht_quant(const void* x, int64_t M, int64_t K, const int6
         const uint32_t ntiles = (uint32_t)(M / NV_TILE) * (uint32_t)p.col_tiles;
         const uint32_t cap = (uint32_t)dev->sms * (uint32_t)dev->amax_blocks_per_sm;
         if (ntiles > 0) launch_nvfp4_amax(pa, ntiles, (int)(ntiles < cap ? ntiles : cap), st);
+        pc.done_per_tile = 0;  // the launch boundary orders the maxima: no counts to wait for
         r = launch_status();
     } else {
         r = launch(pa, na);

@@ -145,8 +145,9 @@ constexpr int NV_WS_HEADER = 4;              // counter, exit count, error, abor
 
 // Workspace words (uint32): [0] claim counter (claims of NV_CLAIM tiles), [1] CTAs finished, [2] sticky
 // error word (cleared by hq_get_error), [3] abort flag of the running call,
-// then amax_row bits [S], amax_col bits [S], amax-pass tiles finished per
-// section [S].  All but [2] are zero between calls.
+// then amax_row bits [S], amax_col bits [S], amax tiles finished per
+// section [S] (the streaming amax kernel counts none).  All but [2] are zero
+// between calls.
 struct NvParams {
     CUtensorMap tmap;   // x as [M/16][16][K] BF16 blocks, 64 x 8 x 16 boxes, 128-byte swizzle
     const uint16_t* x;
@@ -165,6 +166,7 @@ struct NvParams {
     uint32_t multi_claims;  // claims of NV_CLAIM tiles; the claims after them take one tile each
     int finalize;       // last launch of the call: publish amax/sdec, reset ws
     int reset_counter;  // reset the tile counter / exit count at the end
+    uint32_t done_per_tile;  // amax counts wanted per tile: 1 (amax tiles), 0 (after the streaming amax kernel)
     int sec_row0[HQ_MAX_SECTIONS + 1];
     uint32_t seg_start[NV_MAX_SEG + 1];
     uint16_t seg_info[NV_MAX_SEG];  // section | (phase << 15); phase 0 amax, 1 cast

@@ -356,7 +356,7 @@ __device__ __forceinline__ uint32_t nv_prepare(const NvParams& p, StageHdr& h, c
                                       (p.flags & HQ_COLWISE) ? (pre ? ps.pf_ac : p.amax_col[t.s]) : 0.0f);
                 } else if (!g) {
                     const uint32_t* const done = p.ws + NV_WS_HEADER + 2 * p.S + t.s;
-                    const uint32_t target = (uint32_t)(t.ms / NV_TILE) * (uint32_t)p.col_tiles;
+                    const uint32_t target = (uint32_t)(t.ms / NV_TILE) * (uint32_t)p.col_tiles * p.done_per_tile;
                     uint32_t d = ps.pf_s == t.s ? ps.pf : ld_relaxed_u32(done);
                     const bool pf_final = ps.pf_s == t.s && d >= target;  // the prefetched maxima are final
                     uint32_t spins = 0;
@@ -857,42 +857,60 @@ __device__ __forceinline__ void nv_consumer(const NvParams& p, NvShared& sh, con
 
 // ------------------------------------------------------------ amax kernel
 // The section maxima of the two-pass schedule's first launch, streamed
-// through registers (rowwise output without the row RHT): a CTA of 8 warps
-// takes a 128 x 128 tile (grid-stride, in tile order), warp w its rows
-// 16w..16w+15 and lane l the columns 4l..4l+3 of them: 16 eight-byte loads
-// per lane, each warp load instruction one 256-byte row segment, and the
-// next tile's 16 issued before the current one is computed (2 CTAs of 128
-// registers per SM).  The rowwise maximum is taken on the BF16 magnitudes,
-// the columnwise one over the RHT16 outputs of the lane's two column pairs
-// (the functions of the fused kernel's amax tiles).  A tile's maxima and
-// count are published as the amax tiles publish theirs, so the cast launch
-// that follows finds the same workspace state.  (Measured against it: the
-// same without the prefetch at 2-4 CTAs per SM, up to 11 us slower on the
-// grouped MoE call; a TMA-fed version, one CTA per SM with 6 buffers and 16
-// compute warps, 22 us slower.)
+// through registers (rowwise output without the row RHT).  The unit of work
+// is a strip of 16 rows x 128 columns of a tile (8 per tile), taken by one
+// warp: lane l reads columns 4l..4l+3 of the 16 rows (16 eight-byte loads,
+// each warp load instruction one 256-byte row segment), and the next strip's
+// loads are issued before the current one is computed (2 CTAs of 8 warps and
+// 128 registers per SM).  Strips are numbered in tile order (the 8 strips of
+// a tile, then the next tile) and every warp takes one contiguous run of
+// them, on its own: lane 0 keeps the warp's running maxima of its current
+// section and adds them to the section's workspace maxima (two relaxed
+// GPU-scope reductions) when the section changes and at the end, so no warp
+// waits for another and a section's words see a few reductions per warp.  No counts:
+// the cast launch that follows starts after this kernel has finished, which
+// orders every reduction before it, and it reads the maxima as final (zero
+// counts wanted per tile).  The rowwise maximum is taken on the BF16
+// magnitudes, the columnwise one over the RHT16 outputs of the lane's two
+// column pairs (the functions of the fused kernel's amax tiles).  It reads
+// about 4.9 TB/s.  Measured against it on the grouped MoE call: a CTA-wide
+// maximum and a count per tile behind a barrier, the same time; a count with
+// release semantics per strip, 56 us slower (each release waits for the
+// prefetched loads); strips dealt to warps round robin, 27 us slower (a
+// reduction per strip, on the same few words); no prefetch, up to 11 us
+// slower; a TMA-fed version, one CTA per SM with 6 buffers and 16 compute
+// warps, 22 us slower.
 constexpr int NA_THREADS = 256;
+constexpr uint32_t NA_STRIPS = NV_TILE / 16;  // strips per tile
 
 __global__ void __launch_bounds__(NA_THREADS, 2) nvfp4_amax_kernel(const __grid_constant__ NvParams p, uint32_t ntiles) {
-    __shared__ uint32_t acc[2][2];  // [tile parity][rowwise, columnwise] maxima as binary32 bits
     __shared__ int32_t sec_row0[HQ_MAX_SECTIONS + 1];
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     for (int i = tid; i <= p.S; i += NA_THREADS) sec_row0[i] = p.sec_row0[i];
-    if (tid < 4) acc[tid >> 1][tid & 1] = 0u;
     bf16_t sg[16];  // sigma_i as BF16 +-1
 #pragma unroll
     for (int i = 0; i < 16; ++i) sg[i] = ((p.sign_mask >> i) & 1u) ? (bf16_t)0xBF80u : (bf16_t)0x3F80u;
     const bool do_row = p.flags & HQ_ROWWISE, do_col = p.flags & HQ_COLWISE;
     uint32_t* const amax_row_ws = p.ws + NV_WS_HEADER;
     uint32_t* const amax_col_ws = amax_row_ws + p.S;
-    uint32_t* const done_ws = amax_col_ws + p.S;
     const uint32_t ct = (uint32_t)p.col_tiles;
+    const uint32_t nstrips = ntiles * NA_STRIPS, nwarps = gridDim.x * (NA_THREADS / 32);
+    const uint32_t gw = blockIdx.x * (NA_THREADS / 32) + (uint32_t)w;
+    const uint32_t u_begin = (uint32_t)((uint64_t)nstrips * gw / nwarps);
+    const uint32_t u_end = (uint32_t)((uint64_t)nstrips * (gw + 1u) / nwarps);  // this warp's run
     __syncthreads();
-    int s = 0;  // thread 0: section of the current tile (tiles come in increasing order)
-    uint32_t it = 0;
+    int s = 0;  // lane 0: section of the current strip (a warp's strips come in increasing order)
+    uint32_t run_row = 0u, run_col = 0u;  // lane 0: the warp's maxima of section s so far
+    auto flush = [&]() {
+        if (do_row && run_row) red_max_u32(amax_row_ws + s, run_row);
+        if (do_col && run_col) red_max_u32(amax_col_ws + s, run_col);
+        run_row = run_col = 0u;
+    };
     uint32_t na[16], nb[16];
-    auto load = [&](uint32_t t) {
-        const uint32_t rt = t / ct, cti = t - rt * ct;
-        const uint16_t* src = p.x + ((int64_t)rt * NV_TILE + 16 * w) * p.K + (int64_t)cti * NV_TILE + 4 * lane;
+    auto load = [&](uint32_t u) {
+        const uint32_t t = u / NA_STRIPS, rt = t / ct, cti = t - rt * ct;
+        const uint16_t* src = p.x + ((int64_t)rt * NV_TILE + 16 * (u % NA_STRIPS)) * p.K + (int64_t)cti * NV_TILE +
+                              4 * lane;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + i * p.K));
@@ -900,16 +918,16 @@ __global__ void __launch_bounds__(NA_THREADS, 2) nvfp4_amax_kernel(const __grid_
             nb[i] = v.y;
         }
     };
-    if (blockIdx.x < ntiles) load(blockIdx.x);
-    for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
-        const uint32_t rt = t / ct;
+    if (u_begin < u_end) load(u_begin);
+    for (uint32_t u = u_begin; u < u_end; ++u) {
+        const int row0 = (int)((u / NA_STRIPS / ct) * NV_TILE);
         uint32_t wa[16], wb[16];  // row i: columns 4l, 4l + 1 and 4l + 2, 4l + 3
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             wa[i] = na[i];
             wb[i] = nb[i];
         }
-        if (t + gridDim.x < ntiles) load(t + gridDim.x);
+        if (u + 1u < u_end) load(u + 1u);
         uint32_t mrow = 0u;
         float mcol = 0.0f;
         if (do_row) {
@@ -926,21 +944,15 @@ __global__ void __launch_bounds__(NA_THREADS, 2) nvfp4_amax_kernel(const __grid_
         mrow = __reduce_max_sync(0xFFFFFFFFu, mrow);
         const uint32_t mc = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(__fmul_rn(mcol, 0.25f)));
         if (lane == 0) {
-            atomicMax(&acc[it & 1u][0], mrow);
-            atomicMax(&acc[it & 1u][1], mc);
-        }
-        __syncthreads();  // (slot it & 1 is next written two tiles on, after the next barrier)
-        if (tid == 0) {
-            while (sec_row0[s + 1] <= (int)(rt * NV_TILE)) ++s;
-            const uint32_t ar = acc[it & 1u][0], ac = acc[it & 1u][1];
-            acc[it & 1u][0] = 0u;
-            acc[it & 1u][1] = 0u;
-            if (do_row) red_max_u32(amax_row_ws + s, ar);
-            if (do_col) red_max_u32(amax_col_ws + s, ac);
-            // release: a producer that sees the count sees the maxima
-            red_release_add_u32(done_ws + s, 1u);
+            if (sec_row0[s + 1] <= row0) {
+                flush();
+                while (sec_row0[s + 1] <= row0) ++s;
+            }
+            run_row = max(run_row, mrow);
+            run_col = max(run_col, mc);
         }
     }
+    if (lane == 0) flush();
 }
 
 }  // namespace
