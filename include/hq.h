@@ -280,9 +280,9 @@ hq_status hq_group_rht_quant_host(const void *x, int64_t M, int64_t K,
 
 /*
  * hq_group_rht_quant without a caller workspace, for callers that cannot
- * allocate device memory where they quantize (code running while a CUDA
- * graph is captured, plugins whose host framework owns all device memory,
- * allocation-free runtimes).  The paper has no counterpart.
+ * allocate device memory where they quantize (plugins whose host framework
+ * owns all device memory, allocation-free runtimes).  The paper has no
+ * counterpart.
  *
  * Arguments, outputs and errors are those of hq_group_rht_quant without
  * ws / ws_bytes.  The scratch words live in a fixed array inside the library

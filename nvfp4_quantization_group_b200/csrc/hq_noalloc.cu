@@ -2,9 +2,8 @@
 // cast for callers that cannot allocate device memory.
 //
 // Some callers cannot call cudaMalloc (or any allocating routine) at the
-// point where they quantize: code running while a CUDA graph is being
-// captured, plugins whose host framework owns all device memory, or
-// allocation-free inference runtimes.  For them this entry point keeps the
+// point where they quantize: plugins whose host framework owns all device
+// memory, or allocation-free inference runtimes.  For them this entry point keeps the
 // grouped kernel's scratch words (tile counter, per-section amax accumulators
 // and completion counts) in a fixed array of the library itself instead of a
 // caller workspace.  The paper has no counterpart; it is an addition of this

@@ -1,7 +1,7 @@
 """GPU: the allocation-free grouped entry point (hq_group_rht_quant_noalloc).
 
 It exists for callers that cannot allocate device memory where they quantize
-(CUDA graph capture, frameworks that own all device memory): its scratch
+(frameworks that own all device memory): its scratch
 words live in a fixed array inside the library.  Two calls in a row through
 the C ABI must give exactly what hq_group_rht_quant gives with a caller
 workspace (the parity tests compare outputs bit for bit).  This file is
