@@ -348,7 +348,7 @@ def test_interleaved_block_scales_grouped_moe_16384x7168(hq):
 
 
 @pytest.mark.parametrize("flags", [3 | 32 | 64, 1 | 32, 2 | 64, 3 | 64, 1 | 4 | 32, 3 | 4 | 32 | 64 | 8,
-                                   3 | 32 | 64 | 128])
+                                   3 | 32 | 64 | 128, 3 | 32 | 64 | 8])
 def test_stochastic_rounding_matches_oracle(hq, flags):
     """Stochastic rounding is decided by integer comparisons of exact values,
     so the codes must be bit-identical to the oracle's."""
